@@ -1,0 +1,358 @@
+"""Benchmark of one DSpark-style speculative round on B200.
+
+A step is one pass of the whole hot path (draft_sample -> prefix_schedule ->
+verify) over one batch of the serving-shape workload: B=256 requests, K=5
+drafted positions, V=129280, Markov rank 256, bf16 logits, per-request
+temperatures {0.6, 0.8, 1.0}, a cost table with a step at 512 verified tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun every rank runs its own batch (different seed) with no
+collective on the data path (weak scaling); timing is bracketed by a barrier
+and synchronisation, taken with CUDA events, and reduced with MAX over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+from datetime import timedelta
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_decoding_draft_sample_b200 import binding as bn  # noqa: E402
+from speculative_decoding_draft_sample_b200 import workloads as wl  # noqa: E402
+from speculative_decoding_draft_sample_b200.spec_round import (DEVICE_KEYS, SpecRound,  # noqa: E402
+                                                                run_host, to_device)
+
+METRIC = "spec rounds/s & accepted tok/s at B=256,K=5,V=129280; verify HBM GB/s vs peak"
+UNIT = "rounds/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        try:
+            u = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.idx = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            self.idx = vis.split(",")[device_index] if vis else str(device_index)
+        self.proc = None
+        self.path = os.path.join("/tmp", f"dspark_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = max(mx, float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def time_region(fn, stream, iters: int) -> float:
+    """Average ms of fn() over iters runs, CUDA events on ``stream``."""
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(iters):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def cpu_baseline(w: wl.Workload, inp_small, n_req: int, round_id: int):
+    """The fp64 oracle on a bounded sample of the round (n_req requests)."""
+    from oracle import dspark as o
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    reqs = list(range(n_req))
+    part = wl.generate(w, reqs)
+    rid = np.asarray(reqs)
+    oi = dict(target=part["target"].double().numpy(), base=part["base"].double().numpy(),
+              U=inp_small["U"].double().numpy(), W=inp_small["W"].double().numpy(),
+              last_tok=np.asarray(inp_small["last_tok"])[rid],
+              bias_scale=np.asarray(inp_small["bias_scale"], np.float64)[rid],
+              temp=np.asarray(inp_small["temp"], np.float64)[rid],
+              conf_logit=np.asarray(inp_small["conf_logit"], np.float64),
+              pos_temp=np.asarray(inp_small["pos_temp"], np.float64),
+              step_cost=np.asarray(inp_small["step_cost"], np.float64),
+              fixed_cost=float(inp_small["fixed_cost"]), dtype=w.dtype, request_ids=rid)
+    t0 = time.perf_counter()
+    r = o.run_round(oi, wl.PHILOX_SEED, round_id)
+    dt = time.perf_counter() - t0
+    rounds = n_req / w.B
+    return dict(value=rounds / dt, unit=UNIT, cores=int(cores), kind="oracle",
+                sample=f"{n_req} of {w.B} requests of one round (draft with the rank-{w.r} bias, "
+                       f"batch-wide cut, verify), fp64 numpy, scaled by {w.B}/{n_req}",
+                seconds=dt, accepted=int(r["verify"]["a"].sum()))
+
+
+def reference_arm(args, w: wl.Workload):
+    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return
+    small = wl.small_inputs(w)
+    n_req = 4
+    for i in range(args.warmup):
+        cpu_baseline(w, small, 1, 1000 + i)
+    secs = 0.0
+    last = None
+    for i in range(args.steps):
+        last = cpu_baseline(w, small, n_req, i)
+        secs += last["seconds"]
+    value = args.steps * (n_req / w.B) / secs
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                             "sample": last["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = wl.DSPARK5
+    if args.impl == "reference":
+        reference_arm(args, w)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    world, rank, local = dist_setup(args.gpus)
+    hbm, tflops, tflops_sus, peak_kind = peaks()
+
+    # each rank: its own batch (weak scaling), no collective on the data path
+    wr = wl.scaled(w, seed=rank) if rank else w
+    inp = wl.generate(wr)
+    dev = to_device(inp)
+    rnd = SpecRound(w.B, w.K, w.V, w.r, torch.bfloat16)
+    stream = torch.cuda.Stream()
+    round_id = 0
+
+    def step():
+        rnd.run(dev, wl.PHILOX_SEED, round_id, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    torch.cuda.synchronize()
+    code, first = rnd.status(stream)
+    if code:
+        raise RuntimeError(f"device status {code} at request {first}")
+
+    # CUDA graph of the whole round (2K + 2 launches)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            step()
+        stream.synchronize()
+        with torch.cuda.graph(graph, stream=stream):
+            step()
+    torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record(stream)
+    e1.synchronize()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    clk = clocks.stop() if clocks else None
+
+    accepted = int(rnd.accepted.sum().item())
+    emitted = int(rnd.n_emit.sum().item())
+    cut = rnd.cut.cpu().numpy()
+    acc_np = rnd.accepted.cpu().numpy()
+    acc_all = sum_over_ranks(float(accepted), world)
+    emit_all = sum_over_ranks(float(emitted), world)
+    rounds_per_s = world * 1000.0 / ms
+
+    # per-stage times (same stream, CUDA events), each stage alone
+    s_bytes = 2
+    with torch.cuda.stream(stream):
+        ms_draft = time_region(lambda: bn.draft_sample(
+            dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], dev["temp"],
+            wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream),
+            stream, 10)
+        ms_sched = time_region(lambda: bn.prefix_schedule(
+            dev["conf_logit"], dev["pos_temp"], dev["step_cost"], dev["fixed_cost"], bn.CUT_COST,
+            0.0, rnd.cut, rnd.survival, rnd.ws, stream), stream, 20)
+        ms_verify = time_region(lambda: bn.verify(
+            dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
+            round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream), stream, 20)
+    # verify's algorithmic bytes: target rows 0..a_b of every request, plus the
+    # draft row a_b of every request rejected before its cut
+    rej = int((acc_np < cut).sum())
+    verify_bytes = (int((acc_np + 1).sum()) + rej) * w.V * s_bytes
+    verify_gbs = verify_bytes / (ms_verify * 1e-3) / 1e9
+    # draft stage: base in + d out per position, W once per position
+    draft_bytes_pos = 2 * w.B * w.V * s_bytes + w.r * w.V * s_bytes
+    draft_gbs = w.K * draft_bytes_pos / (ms_draft * 1e-3) / 1e9
+    gemm_tflops = 2.0 * w.B * w.r * w.V * w.K / (ms_draft * 1e-3) / 1e12
+
+    # end to end through the public API from pinned host buffers
+    host = to_device(inp, pin=True)
+    out_h = torch.empty_like(rnd.out, device="cpu").pin_memory()
+    n_h = torch.empty_like(rnd.n_emit, device="cpu").pin_memory()
+    h2d = sum(host[k].numel() * host[k].element_size() for k in DEVICE_KEYS)
+    d2h = out_h.numel() * 4 + n_h.numel() * 4
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, stream=stream)
+        barrier(world)
+        e2e_steps = max(3, args.steps // 5)
+        ms_e2e = time_region(lambda: run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h,
+                                              stream=stream), stream, e2e_steps)
+    ms_e2e = max_over_ranks(ms_e2e, world)
+
+    dominant = "verify" if ms_verify >= ms_draft / w.K else "draft"
+    roof = {"kernel": "verify_kernel (dspark_verify)", "bound": "hbm", "achieved": verify_gbs,
+            "peak": hbm, "unit": "GB/s", "frac": verify_gbs / hbm, "traffic": None,
+            "peak_source": f"hbm_gbs of {peak_kind} peaks", "bytes_per_launch": verify_bytes,
+            "launch_ms": ms_verify}
+    line = {
+        "metric": METRIC, "value": rounds_per_s, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded Zipf+noise logits, random Markov factors)",
+        "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
+                   "global_batch": w.B * world, "parallelism": f"replicas{world}",
+                   "l2": "inputs (728 MB) larger than L2 (126 MB); not flushed",
+                   "timing": "CUDA graph of the round, CUDA events, max over ranks"},
+        "accepted_tok_per_s": acc_all * 1000.0 / ms,
+        "emitted_tok_per_s": emit_all * 1000.0 / ms,
+        "accepted_per_round": accepted, "emitted_per_round": emitted,
+        "mean_cut": float(cut.mean()), "mean_accepted": float(acc_np.mean()),
+        "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify},
+        "verify_gbs": verify_gbs, "verify_frac_of_peak": verify_gbs / hbm,
+        "draft_stage": {"gbs": draft_gbs, "bytes_per_position": draft_bytes_pos,
+                        "bias_gemm_tflops": gemm_tflops, "tflops_peak": tflops},
+        "dominant_stage": dominant,
+        "roofline": roof,
+        "e2e": {"value": world * 1000.0 / ms_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+        "gpu_launches": (2 * w.K + 2) * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), 128, 0).items()
+                                if k in ("value", "unit", "cores", "kind", "sample")}
+    del graph
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

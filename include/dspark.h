@@ -1,0 +1,203 @@
+/*
+ * dspark.h — C ABI of the B200 (sm_100a) hot path of one DSpark-style
+ * confidence-scheduled speculative-decoding round:
+ *
+ *   dspark_draft_sample    semi-autoregressive draft: parallel base logits plus
+ *                          a low-rank Markov-head bias, sampled position by position
+ *   dspark_prefix_schedule calibrated confidence, survival products and the
+ *                          early-stopping prefix cut against a cost-per-token table
+ *   dspark_verify          lossless rejection-sampling verification, residual or
+ *                          bonus token, accepted lengths and emitted tokens
+ *
+ * Sources, cited by page title and section:
+ *   [P1] "DSpark turns speculation into a scheduler" (benebsworth.pages.dev)
+ *   [P2] "notes/dspark-deepseek" (skandtandon.pages.dev)
+ *   [P3] "DSpark LLM inference speedup" (probackend.com)
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE pointers, row-major with the vocabulary
+ *     innermost, 16-byte aligned. V must be a multiple of 8.
+ *   - dtype is DSPARK_F32 or DSPARK_BF16 and applies to every logit tensor and
+ *     to the Markov factors U, W. Temperatures, probabilities, confidences and
+ *     costs are always fp32; token ids are int32.
+ *   - The library never allocates or frees device memory. Each call takes a
+ *     caller-owned device workspace of at least dspark_workspace_bytes() bytes;
+ *     its first 256 bytes are a status block that must be zero before first use
+ *     (dspark_clear_status) and that the calls only ever OR bits into.
+ *   - Every call is asynchronous on the given stream (a cudaStream_t; NULL is
+ *     the legacy default stream): no host synchronisation, no device trap.
+ *   - Return value: DSPARK_OK or a negative DSPARK_ERR_* code. Argument errors
+ *     are detected on the host before anything is launched.
+ *   - Data errors found on the device (a token id outside [0, V), a row whose
+ *     logits are NaN, +inf or all -inf, a cut outside [0, K], a negative or NaN
+ *     temperature, a bounded device wait that gave up) set DSPARK_STATUS_* bits
+ *     and the lowest offending request index in the status block; the kernel
+ *     then writes a defined value (token 0, accepted length 0) and carries on.
+ *     dspark_read_status() returns them.
+ *   - Random numbers: Philox4x32-10 (Salmon et al., SC'11), key = seed,
+ *     counter = (request, purpose << 24 | position, lo32(round_id),
+ *     hi32(round_id)), u = (word0 >> 8) * 2^-24; purposes 0 draft, 1 accept,
+ *     2 residual, 3 bonus. A round is fully reproducible from (seed, round_id).
+ */
+#ifndef DSPARK_H
+#define DSPARK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t, so that C callers need no CUDA header. */
+typedef struct CUstream_st* dspark_stream_t;
+
+enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 };
+
+enum {
+  DSPARK_OK = 0,
+  DSPARK_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misalignment      */
+  DSPARK_ERR_UNSUPPORTED = -2,  /* dtype, shape or device not supported      */
+  DSPARK_ERR_CUDA = -3,         /* a CUDA launch or runtime call failed      */
+  DSPARK_ERR_WORKSPACE = -4,    /* workspace smaller than the query's answer */
+  DSPARK_ERR_TIMEOUT = -5       /* reported by dspark_read_status only       */
+};
+
+enum { DSPARK_OP_DRAFT = 0, DSPARK_OP_SCHEDULE = 1, DSPARK_OP_VERIFY = 2 };
+
+/* Prefix-cut modes of dspark_prefix_schedule. */
+enum { DSPARK_CUT_COST = 0, DSPARK_CUT_THRESHOLD = 1, DSPARK_CUT_NONE = 2 };
+
+/* Bits of the device status word. */
+#define DSPARK_STATUS_BAD_TOKEN 0x1u /* token id outside [0, V)                 */
+#define DSPARK_STATUS_BAD_ROW 0x2u   /* NaN / +inf / all -inf logits in a row    */
+#define DSPARK_STATUS_BAD_CUT 0x4u   /* cut outside [0, K]                       */
+#define DSPARK_STATUS_BAD_TEMP 0x8u  /* temperature negative or NaN             */
+#define DSPARK_STATUS_TIMEOUT 0x10u  /* a bounded device wait gave up           */
+
+/*
+ * Workspace bytes needed by operation `op` (DSPARK_OP_*) for these sizes
+ * (r is ignored except by DSPARK_OP_DRAFT). Pure host function. Returns 0 for
+ * unsupported arguments. One workspace of the largest size may serve all three
+ * operations on one stream.
+ */
+size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype);
+
+/*
+ * Draft sampling with the Markov head, K positions in turn.
+ * [P1] "DSpark's semi-autoregressive compromise" (parallel base logits plus a
+ * prefix-dependent transition bias from the previous sampled token);
+ * [P3] "The Semi-Autoregressive Trick" (low-rank Markov head, rank 256).
+ *
+ * For k = 1..K and every request b:
+ *   bias     = bias_scale[b] * U[x_{b,k-1}, :] @ W          (fp32 accumulation)
+ *   d[b,k-1] = round_dtype(base[b,k-1] + bias)              (stored logits)
+ *   x[b,k-1] ~ softmax(d[b,k-1] / temp[b]) by inverse CDF in index order with
+ *              u = Philox(seed, b, k, purpose 0, round_id); argmax (lowest index
+ *              on ties) when temp[b] == 0
+ *   q_lse    = log-sum-exp of d/temp; q_tok = q(x). For greedy requests
+ *              q_tok = 1 and q_lse = max d.
+ * with x_{b,0} = last_tok[b] (the last committed token).
+ *
+ *   base       [B, K, V] dtype   parallel drafter's base logits
+ *   U          [V, r]    dtype   Markov factor, row per previous token
+ *   W          [r, V]    dtype   Markov factor
+ *   bias_scale [B] f32 or NULL   per-request multiplier of the bias (NULL: 1)
+ *   last_tok   [B] i32           last committed token of each request
+ *   temp       [B] f32           sampling temperature, 0 = greedy
+ *   x          [B, K] i32  out   drafted tokens
+ *   d          [B, K, V] dtype out  stored draft logits (verification uses them)
+ *   q_lse      [B, K] f32  out   log normaliser of d/temp
+ *   q_tok      [B, K] f32  out   draft probability of each drafted token
+ * Limits: 1 <= B <= 65535, 1 <= K <= 64, 8 <= V < 2^24, 1 <= r <= 1024;
+ * bf16 additionally needs r % 16 == 0.
+ */
+int dspark_draft_sample(const void* base, const void* U, const void* W,
+                        const float* bias_scale, const int32_t* last_tok,
+                        const float* temp, int B, int K, int V, int r, int dtype,
+                        uint64_t seed, uint64_t round_id, int32_t* x, void* d,
+                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
+                        dspark_stream_t stream);
+
+/*
+ * Calibrated confidence, survival and the prefix cut.
+ * [P1] "Confidence is a serving primitive" (c_k, survival product
+ * P(prefix 1:k survives) = prod_{i<=k} c_i, Sequential Temperature Scaling,
+ * hardware-aware prefix scheduler, static threshold as the rule it departs
+ * from); [P1] "The speculative loop" (latency equation, the objective);
+ * [P3] "The Real Innovation: Confidence-Scheduled Verification" (early stop).
+ *
+ *   c[b,k] = sigmoid(conf_logit[b,k] / pos_temp[k]),  S[b,k] = prod_{i<=k} c[b,i]
+ * mode DSPARK_CUT_COST: every request verifies one slot for its correction or
+ *   bonus token; verifying n tokens costs fixed_cost + step_cost[0] + ... +
+ *   step_cost[n-1]. Drafts are visited by descending S (ties: smaller k, then
+ *   smaller b) and admitted while S_j * C_{j-1} >= A_{j-1} * step_cost[B+j-1]
+ *   (A = B + admitted S, C = current cost, j 1-based); the first failure stops
+ *   the walk. cut[b] = admitted drafts of request b (a prefix of its block).
+ * mode DSPARK_CUT_THRESHOLD: cut[b] = #{k : S[b,k] >= threshold}.
+ * mode DSPARK_CUT_NONE: cut[b] = K.
+ * Computed in fp64 on the device; survival is returned rounded to fp32.
+ *
+ *   conf_logit [B, K] f32, pos_temp [K] f32 (> 0), step_cost [B*(K+1)] f32
+ *   cut [B] i32 out, survival [B, K] f32 out
+ * Limits: 1 <= K <= 64; the cost rule needs B*K <= 8192 (one CTA sorts all
+ * drafts), the other modes take any B >= 1.
+ */
+int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp,
+                           const float* step_cost, float fixed_cost, int B, int K,
+                           int mode, float threshold, int32_t* cut,
+                           float* survival, void* ws, size_t ws_bytes,
+                           dspark_stream_t stream);
+
+/*
+ * Lossless verification of the first cut[b] drafts of every request.
+ * [P1] intro and "Caveats" (accept the longest valid prefix, correct at the
+ * first rejection; lossless only with the proper acceptance rule); [P2]
+ * "Sources" (the rule of "Fast Inference from Transformers via Speculative
+ * Decoding"); [P3] "Speculative Decoding in Two Sentences" (plus one bonus
+ * token; the target distribution is preserved exactly).
+ *
+ * Target row j (0-based) scores draft token j+1; row cut[b] gives the bonus.
+ * For k = 1..cut[b]: p = softmax(target[b,k-1] / temp[b]); accept x[b,k-1]
+ * iff Philox(seed, b, k, purpose 1, round_id) < p(x) / q_tok[b,k-1]; stop at
+ * the first rejection. accepted[b] = a. If a < cut[b]: y ~ norm(max(0, p - q))
+ * over target row a and q = softmax(d[b,a] / temp[b]) (purpose 2, position
+ * a+1; p itself if the residual is exactly zero). Else y ~ p of target row
+ * cut[b] (purpose 3, position a+1). Greedy requests (temp 0) accept iff
+ * x == argmax of the target row and emit argmax of target row a.
+ * out[b] = x[b,0..a-1], y, then -1 up to K+1 entries; n_emit[b] = a + 1.
+ * Only target rows 0..a and draft row a are read.
+ *
+ *   target [B, K+1, V] dtype, d [B, K, V] dtype, x [B, K] i32,
+ *   q_tok [B, K] f32, cut [B] i32 or NULL (all K), temp [B] f32
+ *   accepted [B] i32 out, out [B, K+1] i32 out, n_emit [B] i32 out
+ * Limits: 1 <= B <= 65535, 1 <= K <= 64, 8 <= V < 2^24.
+ */
+int dspark_verify(const void* target, const void* d, const int32_t* x,
+                  const float* q_tok, const int32_t* cut, const float* temp,
+                  int B, int K, int V, int dtype, uint64_t seed,
+                  uint64_t round_id, int32_t* accepted, int32_t* out,
+                  int32_t* n_emit, void* ws, size_t ws_bytes,
+                  dspark_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads the status block of `ws` into *code (OR of
+ * DSPARK_STATUS_* bits) and *first_bad_request (-1 if none), then clears it.
+ * Either output pointer may be NULL.
+ */
+int dspark_read_status(void* ws, dspark_stream_t stream, uint32_t* code,
+                       int32_t* first_bad_request);
+
+/* Zeroes the status block of `ws` asynchronously on `stream`. */
+int dspark_clear_status(void* ws, dspark_stream_t stream);
+
+/* Static description of a DSPARK_OK / DSPARK_ERR_* return code. */
+const char* dspark_status_string(int code);
+
+/* ABI version of this header: (major << 16) | minor. */
+int dspark_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSPARK_H */

@@ -252,8 +252,14 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
         if teacher is not None:
             tx = np.asarray(teacher["x"][:, k - 1], np.int64)
             take = st["x_flag"] & (tx != st["x"])
-            forced += int(take.sum())
-            st["x"] = np.where(take, tx, st["x"])
+            if take.any():
+                # the adopted token's own draft probability q(x)
+                forced += int(take.sum())
+                st["x"] = np.where(take, tx, st["x"])
+                rows = np.nonzero(take & (tau > 0))[0]
+                if len(rows):
+                    w, Z, _ = softmax_parts(st["d"][rows], tau[rows])
+                    st["q_tok"][rows] = w[np.arange(len(rows)), st["x"][rows]] / Z
         d[:, k - 1] = st["d"]
         x[:, k - 1], q_lse[:, k - 1], q_tok[:, k - 1] = st["x"], st["q_lse"], st["q_tok"]
         x_flag[:, k - 1] = st["x_flag"]

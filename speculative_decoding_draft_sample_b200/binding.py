@@ -1,0 +1,162 @@
+"""Thin Python binding of libdspark.so (include/dspark.h), via ctypes.
+
+Argument marshalling only: every function takes PyTorch CUDA tensors, checks
+that they are contiguous and on the device, and passes their data pointers and
+sizes to the C entry point of the same name. All arithmetic happens in the
+library's kernels; there is no fallback path. If the library is missing, every
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdspark.so")
+
+F32, BF16 = 0, 1
+OP_DRAFT, OP_SCHEDULE, OP_VERIFY = 0, 1, 2
+CUT_COST, CUT_THRESHOLD, CUT_NONE = 0, 1, 2
+STATUS_BAD_TOKEN, STATUS_BAD_ROW, STATUS_BAD_CUT, STATUS_BAD_TEMP, STATUS_TIMEOUT = 1, 2, 4, 8, 16
+
+_lib = None
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int
+_u64 = ctypes.c_uint64
+_sz = ctypes.c_size_t
+_f = ctypes.c_float
+
+SIGNATURES = {
+    "dspark_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
+    "dspark_draft_sample": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
+                                 _p, _p, _p, _p, _p, _sz, _p]),
+    "dspark_prefix_schedule": (_i, [_p, _p, _p, _f, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
+    "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
+                           _p, _sz, _p]),
+    "dspark_read_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32),
+                                ctypes.POINTER(ctypes.c_int32)]),
+    "dspark_clear_status": (_i, [_p, _p]),
+    "dspark_status_string": (ctypes.c_char_p, [_i]),
+    "dspark_version": (_i, []),
+}
+
+
+class DSparkError(RuntimeError):
+    pass
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise DSparkError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m speculative_decoding_draft_sample_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        msg = lib().dspark_status_string(rc).decode()
+        raise DSparkError(f"{what} failed ({rc}): {msg}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise DSparkError(f"unsupported logit dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise DSparkError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise DSparkError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise DSparkError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def workspace_bytes(op: int, B: int, K: int, V: int, r: int, dtype: int) -> int:
+    return int(lib().dspark_workspace_bytes(op, B, K, V, r, dtype))
+
+
+def version() -> int:
+    return int(lib().dspark_version())
+
+
+def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: int,
+                 x, d, q_lse, q_tok, ws, stream=None) -> None:
+    """dspark_draft_sample: base [B,K,V], U [V,r], W [r,V] -> x, d, q_lse, q_tok."""
+    B, K, V = base.shape
+    r = U.shape[1]
+    dt = _dtype_code(base)
+    rc = lib().dspark_draft_sample(
+        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
+        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
+        _ptr(temp, "temp", torch.float32), B, K, V, r, dt, seed, round_id,
+        _ptr(x, "x", torch.int32), _ptr(d, "d", base.dtype), _ptr(q_lse, "q_lse", torch.float32),
+        _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream))
+    _check(rc, "dspark_draft_sample")
+
+
+def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: int,
+                    threshold: float, cut, survival, ws, stream=None) -> None:
+    """dspark_prefix_schedule: conf_logit [B,K], pos_temp [K], step_cost [B(K+1)] -> cut, survival."""
+    B, K = conf_logit.shape
+    rc = lib().dspark_prefix_schedule(
+        _ptr(conf_logit, "conf_logit", torch.float32), _ptr(pos_temp, "pos_temp", torch.float32),
+        _ptr(step_cost, "step_cost", torch.float32), float(fixed_cost), B, K, mode,
+        float(threshold), _ptr(cut, "cut", torch.int32), _ptr(survival, "survival", torch.float32),
+        _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "dspark_prefix_schedule")
+
+
+def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out, n_emit,
+           ws, stream=None) -> None:
+    """dspark_verify: target [B,K+1,V], d [B,K,V], x, q_tok [B,K], cut [B] -> accepted, out, n_emit."""
+    B, K1, V = target.shape
+    dt = _dtype_code(target)
+    rc = lib().dspark_verify(
+        _ptr(target, "target"), _ptr(d, "d", target.dtype), _ptr(x, "x", torch.int32),
+        _ptr(q_tok, "q_tok", torch.float32), _ptr(cut, "cut", torch.int32),
+        _ptr(temp, "temp", torch.float32), B, K1 - 1, V, dt, seed, round_id,
+        _ptr(accepted, "accepted", torch.int32), _ptr(out, "out", torch.int32),
+        _ptr(n_emit, "n_emit", torch.int32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream))
+    _check(rc, "dspark_verify")
+
+
+def read_status(ws, stream=None) -> Tuple[int, int]:
+    """(status bits, first offending request or -1); synchronises and clears."""
+    code = ctypes.c_uint32(0)
+    first = ctypes.c_int32(-1)
+    rc = lib().dspark_read_status(_ptr(ws, "ws"), _stream(stream), ctypes.byref(code),
+                                  ctypes.byref(first))
+    _check(rc, "dspark_read_status")
+    return int(code.value), int(first.value)
+
+
+def clear_status(ws, stream=None) -> None:
+    _check(lib().dspark_clear_status(_ptr(ws, "ws"), _stream(stream)), "dspark_clear_status")

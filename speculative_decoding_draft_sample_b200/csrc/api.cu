@@ -1,0 +1,202 @@
+// C ABI of libdspark.so: argument checks, workspace layout and launches.
+// Declarations and the contract of every entry point are in include/dspark.h.
+#include <climits>
+#include <cstring>
+
+#include "common.cuh"
+#include "draft.cuh"
+#include "schedule.cuh"
+#include "verify.cuh"
+
+using namespace dspark;
+
+namespace {
+
+constexpr int kAbiVersion = (1 << 16) | 0;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline int nchunks(int V) { return (V + kChunk - 1) / kChunk; }
+
+bool shape_ok(int B, int K, int V, int dtype) {
+  if (dtype != DSPARK_F32 && dtype != DSPARK_BF16) return false;
+  if (B < 1 || B > 65535 || K < 1 || K > 64) return false;
+  if (V < 8 || V >= (1 << 24) || V % 8 != 0) return false;
+  return true;
+}
+
+// The fatbin carries sm_100a code only.
+int device_check(int* num_sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return DSPARK_ERR_CUDA;
+  if (major != 10 || minor != 0) return DSPARK_ERR_UNSUPPORTED;
+  if (num_sms) *num_sms = sms;
+  return DSPARK_OK;
+}
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int dspark_version(void) { return kAbiVersion; }
+
+const char* dspark_status_string(int code) {
+  switch (code) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_ERR_INVALID_ARG: return "invalid argument (null pointer, size or alignment)";
+    case DSPARK_ERR_UNSUPPORTED: return "unsupported dtype, shape or device";
+    case DSPARK_ERR_CUDA: return "CUDA launch or runtime error";
+    case DSPARK_ERR_WORKSPACE: return "workspace too small";
+    case DSPARK_ERR_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+  }
+}
+
+size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype) {
+  switch (op) {
+    case DSPARK_OP_DRAFT:
+      if (!shape_ok(B, K, V, dtype) || r < 1 || r > 1024) return 0;
+      return kStatusBytes + round_up((size_t)B * nchunks(V) * sizeof(float2), 256);
+    case DSPARK_OP_SCHEDULE:
+      if (B < 1 || K < 1 || K > 64) return 0;
+      return kStatusBytes;
+    case DSPARK_OP_VERIFY:
+      if (!shape_ok(B, K, V, dtype)) return 0;
+      return kStatusBytes;
+    default:
+      return 0;
+  }
+}
+
+int dspark_clear_status(void* ws, dspark_stream_t stream) {
+  if (!ws) return DSPARK_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream));
+}
+
+int dspark_read_status(void* ws, dspark_stream_t stream, uint32_t* code, int32_t* first_bad) {
+  if (!ws) return DSPARK_ERR_INVALID_ARG;
+  Status h;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (code) *code = h.code;
+  if (first_bad) *first_bad = (h.first_bad_enc == 0) ? -1 : INT_MAX - h.first_bad_enc;
+  return dspark_clear_status(ws, stream);
+}
+
+int dspark_draft_sample(const void* base, const void* U, const void* W, const float* bias_scale,
+                        const int32_t* last_tok, const float* temp, int B, int K, int V, int r,
+                        int dtype, uint64_t seed, uint64_t round_id, int32_t* x, void* d,
+                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
+                        dspark_stream_t stream) {
+  if (!base || !U || !W || !last_tok || !temp || !x || !d || !q_lse || !q_tok || !ws)
+    return DSPARK_ERR_INVALID_ARG;
+  if (!shape_ok(B, K, V, dtype) || r < 1 || r > 1024) return DSPARK_ERR_INVALID_ARG;
+  if (dtype == DSPARK_BF16 && r % 16 != 0) return DSPARK_ERR_UNSUPPORTED;
+  if (!aligned16(base) || !aligned16(U) || !aligned16(W) || !aligned16(d) || !aligned16(ws))
+    return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_DRAFT, B, K, V, r, dtype))
+    return DSPARK_ERR_WORKSPACE;
+  int sms = 0;
+  if (int e = device_check(&sms)) return e;
+  DraftArgs a;
+  a.base = base;
+  a.U = U;
+  a.W = W;
+  a.bias_scale = bias_scale;
+  a.last_tok = last_tok;
+  a.temp = temp;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.r = r;
+  a.dtype = dtype;
+  a.seed = seed;
+  a.round_id = round_id;
+  a.x = x;
+  a.d = d;
+  a.q_lse = q_lse;
+  a.q_tok = q_tok;
+  a.status = static_cast<Status*>(ws);
+  a.partials = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
+  a.nchunk = nchunks(V);
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int k = 1; k <= K; ++k) {
+    cudaError_t e = draft_logits_simt_launch(a, k, s);
+    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  return DSPARK_OK;
+}
+
+int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp, const float* step_cost,
+                           float fixed_cost, int B, int K, int mode, float threshold, int32_t* cut,
+                           float* survival, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (!conf_logit || !pos_temp || !cut || !survival || !ws) return DSPARK_ERR_INVALID_ARG;
+  if (mode != DSPARK_CUT_COST && mode != DSPARK_CUT_THRESHOLD && mode != DSPARK_CUT_NONE)
+    return DSPARK_ERR_INVALID_ARG;
+  if (mode == DSPARK_CUT_COST && !step_cost) return DSPARK_ERR_INVALID_ARG;
+  if (B < 1 || K < 1 || K > 64) return DSPARK_ERR_INVALID_ARG;
+  if (mode == DSPARK_CUT_COST && (long long)B * K > kMaxScheduleItems) return DSPARK_ERR_UNSUPPORTED;
+  if (!aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_SCHEDULE, B, K, 8, 1, DSPARK_F32))
+    return DSPARK_ERR_WORKSPACE;
+  if (int e = device_check(nullptr)) return e;
+  SchedArgs a;
+  a.conf_logit = conf_logit;
+  a.pos_temp = pos_temp;
+  a.step_cost = step_cost;
+  a.fixed_cost = fixed_cost;
+  a.B = B;
+  a.K = K;
+  a.mode = mode;
+  a.threshold = threshold;
+  a.cut = cut;
+  a.survival = survival;
+  a.status = static_cast<Status*>(ws);
+  return cuda_status(prefix_schedule_launch(a, (cudaStream_t)stream));
+}
+
+int dspark_verify(const void* target, const void* d, const int32_t* x, const float* q_tok,
+                  const int32_t* cut, const float* temp, int B, int K, int V, int dtype,
+                  uint64_t seed, uint64_t round_id, int32_t* accepted, int32_t* out,
+                  int32_t* n_emit, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (!target || !d || !x || !q_tok || !temp || !accepted || !out || !n_emit || !ws)
+    return DSPARK_ERR_INVALID_ARG;
+  if (!shape_ok(B, K, V, dtype)) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(target) || !aligned16(d) || !aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_VERIFY, B, K, V, 1, dtype))
+    return DSPARK_ERR_WORKSPACE;
+  int sms = 0;
+  if (int e = device_check(&sms)) return e;
+  VerifyArgs a;
+  a.target = target;
+  a.d = d;
+  a.x = x;
+  a.q_tok = q_tok;
+  a.cut = cut;
+  a.temp = temp;
+  a.B = B;
+  a.K = K;
+  a.V = V;
+  a.dtype = dtype;
+  a.seed = seed;
+  a.round_id = round_id;
+  a.accepted = accepted;
+  a.out = out;
+  a.n_emit = n_emit;
+  a.status = static_cast<Status*>(ws);
+  const int C = verify_cluster_size(B, V, dtype, sms);
+  return cuda_status(verify_launch(a, C, (cudaStream_t)stream));
+}
+
+}  // extern "C"

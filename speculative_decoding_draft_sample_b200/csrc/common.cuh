@@ -1,0 +1,143 @@
+// Shared device helpers of the speculative-round kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+// Status block at the start of every workspace.
+struct Status {
+  unsigned int code;       // OR of DSPARK_STATUS_* bits
+  int first_bad_enc;       // INT_MAX - lowest offending request; 0 when none
+  unsigned int pad[62];
+};
+static_assert(sizeof(Status) == 256, "status block is 256 bytes");
+constexpr size_t kStatusBytes = 256;
+
+__device__ __forceinline__ void report(Status* st, unsigned int bits, int request) {
+  atomicOr(&st->code, bits);
+  atomicMax(&st->first_bad_enc, 0x7fffffff - request);
+}
+
+// log2(e): every sampling kernel works with z = logit * log2(e) / temperature,
+// so that exp2 gives the unnormalised softmax weight.
+constexpr float kLog2e = 1.44269504088896340736f;
+
+// Bounded spin limit for every device-side wait (mbarrier polls).
+constexpr long long kSpinLimit = 1ll << 26;
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+// as 1, 2, 3", SC'11): ten rounds of two 32x32->64 multiplies whose halves are
+// mixed with the other counter words and the key; the key is bumped by the
+// Weyl constants between rounds.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint32_t c2,
+                                                 uint32_t c3, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int i = 0; i < 10; ++i) {
+    if (i) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0, n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  return c0;
+}
+
+enum Purpose : uint32_t { kDraft = 0, kAccept = 1, kResidual = 2, kBonus = 3 };
+
+// The round's 24-bit uniform for (request, position, purpose); exact in fp32.
+__device__ __forceinline__ float uniform24(uint64_t seed, uint64_t round_id, uint32_t request,
+                                           uint32_t position, uint32_t purpose) {
+  const uint32_t w = philox_word0(request, (purpose << 24) | position, (uint32_t)round_id,
+                                  (uint32_t)(round_id >> 32), (uint32_t)seed,
+                                  (uint32_t)(seed >> 32));
+  return (float)(w >> 8) * (1.0f / 16777216.0f);
+}
+
+// ---------------------------------------------------------------------------
+// element access
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+template <int DT>
+struct Elem;
+
+template <>
+struct Elem<DSPARK_F32> {
+  using T = float;
+  static constexpr int kBytes = 4;
+  __device__ __forceinline__ static float load(const T* p, long long i) { return p[i]; }
+  __device__ __forceinline__ static T store_round(float v) { return v; }
+  __device__ __forceinline__ static float to_float(T v) { return v; }
+};
+
+template <>
+struct Elem<DSPARK_BF16> {
+  using T = uint16_t;
+  static constexpr int kBytes = 2;
+  __device__ __forceinline__ static float load(const T* p, long long i) {
+    return bf16_bits_to_float(p[i]);
+  }
+  __device__ __forceinline__ static T store_round(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  }
+  __device__ __forceinline__ static float to_float(T v) { return bf16_bits_to_float(v); }
+};
+
+// A row is unusable for sampling when it holds NaN or +inf, or is all -inf.
+__device__ __forceinline__ bool bad_logit(float v) { return v != v || v == __int_as_float(0x7f800000); }
+
+// ---------------------------------------------------------------------------
+// reductions
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// (value, index) max with the lowest index on ties.
+__device__ __forceinline__ void argmax_merge(float& v, int& i, float v2, int i2) {
+  if (v2 > v || (v2 == v && i2 < i)) {
+    v = v2;
+    i = i2;
+  }
+}
+__device__ __forceinline__ void warp_argmax(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float v2 = __shfl_xor_sync(0xffffffffu, v, o);
+    const int i2 = __shfl_xor_sync(0xffffffffu, i, o);
+    argmax_merge(v, i, v2, i2);
+  }
+}
+// Inclusive prefix sum over a warp (lane order).
+__device__ __forceinline__ float warp_inclusive_scan(float v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+}  // namespace dspark

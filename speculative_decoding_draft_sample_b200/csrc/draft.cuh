@@ -1,0 +1,33 @@
+// Internal interface of the draft-stage kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+// Vocabulary entries per chunk partial (one online-softmax partial per
+// (request, chunk)); the sampler rescans one chunk to place its draw.
+constexpr int kChunk = 256;
+
+struct DraftArgs {
+  const void* base;        // [B, K, V]
+  const void* U;           // [V, r]
+  const void* W;           // [r, V]
+  const float* bias_scale; // [B] or null
+  const int32_t* last_tok; // [B]
+  const float* temp;       // [B]
+  int B, K, V, r, dtype;
+  uint64_t seed, round_id;
+  int32_t* x;              // [B, K]
+  void* d;                 // [B, K, V]
+  float* q_lse;            // [B, K]
+  float* q_tok;            // [B, K]
+  float2* partials;        // [B, nchunk] in the workspace
+  int nchunk;
+  Status* status;
+};
+
+cudaError_t draft_logits_simt_launch(const DraftArgs& a, int k, cudaStream_t s);
+cudaError_t draft_sample_launch(const DraftArgs& a, int k, cudaStream_t s);
+
+}  // namespace dspark

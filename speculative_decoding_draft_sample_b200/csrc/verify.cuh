@@ -1,0 +1,31 @@
+// Internal interface of the verification kernel.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+struct VerifyArgs {
+  const void* target;     // [B, K+1, V]
+  const void* d;          // [B, K, V]
+  const int32_t* x;       // [B, K]
+  const float* q_tok;     // [B, K]
+  const int32_t* cut;     // [B] or null
+  const float* temp;      // [B]
+  int B, K, V, dtype;
+  uint64_t seed, round_id;
+  int32_t* accepted;      // [B]
+  int32_t* out;           // [B, K+1]
+  int32_t* n_emit;        // [B]
+  Status* status;
+  int slice;              // vocabulary entries per CTA (multiple of 8)
+  size_t slice_bytes_padded;
+};
+
+// CTAs per request (the cluster size) for this batch shape.
+int verify_cluster_size(int B, int V, int dtype, int num_sms);
+// Dynamic shared memory of one CTA; also returns the slice length and its padded bytes.
+size_t verify_smem_bytes(int V, int dtype, int C, int* slice, size_t* slice_padded);
+cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s);
+
+}  // namespace dspark

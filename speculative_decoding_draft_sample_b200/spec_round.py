@@ -1,0 +1,85 @@
+"""One speculative round on the device: draft_sample -> prefix_schedule -> verify.
+
+``SpecRound`` owns the round's output buffers and one workspace (PyTorch
+allocations: device memory is PyTorch's job here) and issues the three C-ABI
+calls on one stream. ``run_host`` is the end-to-end form: inputs in pinned host
+memory are copied in, the round runs, and the emitted tokens come back.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import binding as bn
+
+
+class SpecRound:
+    def __init__(self, B: int, K: int, V: int, r: int, dtype: torch.dtype = torch.bfloat16,
+                 device: str = "cuda"):
+        self.B, self.K, self.V, self.r = B, K, V, r
+        self.dtype = dtype
+        dev = torch.device(device)
+        code = bn.F32 if dtype == torch.float32 else bn.BF16
+        i32 = dict(dtype=torch.int32, device=dev)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.x = torch.empty((B, K), **i32)
+        self.d = torch.empty((B, K, V), dtype=dtype, device=dev)
+        self.q_lse = torch.empty((B, K), **f32)
+        self.q_tok = torch.empty((B, K), **f32)
+        self.cut = torch.empty((B,), **i32)
+        self.survival = torch.empty((B, K), **f32)
+        self.accepted = torch.empty((B,), **i32)
+        self.out = torch.empty((B, K + 1), **i32)
+        self.n_emit = torch.empty((B,), **i32)
+        nbytes = max(bn.workspace_bytes(op, B, K, V, r, code)
+                     for op in (bn.OP_DRAFT, bn.OP_SCHEDULE, bn.OP_VERIFY))
+        if nbytes == 0:
+            raise bn.DSparkError(f"unsupported round shape B={B} K={K} V={V} r={r}")
+        self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
+
+    def run(self, inp: Dict[str, torch.Tensor], seed: int, round_id: int,
+            mode: int = bn.CUT_COST, threshold: float = 0.0, stream=None) -> None:
+        """Issues the round on ``stream`` (no host synchronisation)."""
+        bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
+                        inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
+                        self.ws, stream)
+        bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
+                           float(inp["fixed_cost"]), mode, threshold, self.cut, self.survival,
+                           self.ws, stream)
+        bn.verify(inp["target"], self.d, self.x, self.q_tok, self.cut, inp["temp"], seed,
+                  round_id, self.accepted, self.out, self.n_emit, self.ws, stream)
+
+    def status(self, stream=None):
+        return bn.read_status(self.ws, stream)
+
+
+DEVICE_KEYS = ("base", "target", "U", "W", "bias_scale", "last_tok", "temp", "conf_logit",
+               "pos_temp", "step_cost")
+
+
+def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -> Dict[str, object]:
+    """Device (or pinned host) copies of a workload's tensors (numpy arrays become tensors)."""
+    out: Dict[str, object] = {}
+    for k in DEVICE_KEYS:
+        v = inp[k]
+        t = v if isinstance(v, torch.Tensor) else torch.from_numpy(v)
+        if k == "last_tok":
+            t = t.to(torch.int32)
+        elif t.dtype == torch.float64:
+            t = t.float()
+        t = t.contiguous()
+        out[k] = t.pin_memory() if pin else t.to(device, non_blocking=False)
+    out["fixed_cost"] = float(inp["fixed_cost"])
+    return out
+
+
+def run_host(rnd: SpecRound, host: Dict[str, object], dev: Dict[str, object], seed: int,
+             round_id: int, out_host: torch.Tensor, n_emit_host: torch.Tensor,
+             mode: int = bn.CUT_COST, stream=None) -> None:
+    """End to end from pinned host buffers: H2D copies, the round, D2H of the tokens."""
+    for k in DEVICE_KEYS:
+        dev[k].copy_(host[k], non_blocking=True)
+    rnd.run(dev, seed, round_id, mode, stream=stream)
+    out_host.copy_(rnd.out, non_blocking=True)
+    n_emit_host.copy_(rnd.n_emit, non_blocking=True)

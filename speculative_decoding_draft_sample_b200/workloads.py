@@ -18,6 +18,7 @@ and bit-identically (used to check sampled requests of the large cases).
 from __future__ import annotations
 
 import dataclasses
+import os
 from typing import Dict, List, Optional, Sequence
 
 import numpy as np
@@ -214,9 +215,19 @@ def generate(w: Workload, requests: Optional[List[int]] = None) -> Dict[str, obj
     tdt = torch.float32 if w.dtype == F32 else torch.bfloat16
     target = torch.empty((len(reqs), w.K + 1, w.V), dtype=tdt)
     base = torch.empty((len(reqs), w.K, w.V), dtype=tdt)
-    for i, b in enumerate(reqs):
+
+    def fill(i_b):
+        i, b = i_b
         t, bs = request_rows(w, b, zl, kinds)
         target[i] = t
         base[i] = bs
+
+    if len(reqs) >= 16:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, enumerate(reqs)))
+    else:
+        for ib in enumerate(reqs):
+            fill(ib)
     out.update(target=target, base=base, requests=reqs)
     return out

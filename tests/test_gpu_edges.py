@@ -1,0 +1,139 @@
+"""Degenerate cases, device status reporting and argument errors of the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from parity import SEED, check_round, run_gpu
+from speculative_decoding_draft_sample_b200 import binding as bn
+from speculative_decoding_draft_sample_b200 import workloads as wl
+from speculative_decoding_draft_sample_b200.spec_round import SpecRound, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _small(**kw):
+    base = dict(name="edge", B=16, V=2048)
+    base.update(kw)
+    return wl.scaled(wl.DSPARK5, **base)
+
+
+def test_identical_draft_full_acceptance_and_bonus(cuda_ok):
+    w = _small(identical_frac=1.0)
+    inp = wl.generate(w)
+    rnd, _ = run_gpu(w, inp, 2, bn.CUT_NONE)
+    check_round(w, inp, rnd, list(range(w.B)), 2, bn.CUT_NONE)
+    assert np.all(rnd.accepted.cpu().numpy() == w.K)
+    assert np.all(rnd.n_emit.cpu().numpy() == w.K + 1)
+
+
+def test_independent_draft_residual_path(cuda_ok):
+    w = _small(independent_frac=1.0)
+    inp = wl.generate(w)
+    rnd, _ = run_gpu(w, inp, 4, bn.CUT_NONE)
+    check_round(w, inp, rnd, list(range(w.B)), 4, bn.CUT_NONE)
+    assert rnd.accepted.float().mean().item() < 0.5
+
+
+def test_greedy_exact_match(cuda_ok):
+    w = _small(greedy_frac=1.0, B=32)
+    inp = wl.generate(w)
+    rnd, _ = run_gpu(w, inp, 0, bn.CUT_NONE)
+    check_round(w, inp, rnd, list(range(w.B)), 0, bn.CUT_NONE)
+    # greedy drafts are argmax d, greedy emission argmax of the target row
+    d = rnd.d.float().cpu()
+    assert torch.equal(rnd.x.cpu().long(), d.argmax(dim=2))
+
+
+def test_zero_bias_equals_parallel_drafter(cuda_ok):
+    """bias_scale = 0 gives d == round(base) exactly, and W = 0 the same draws."""
+    w = _small(B=8)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    dev["bias_scale"] = torch.zeros(w.B, device="cuda")
+    rnd = SpecRound(w.B, w.K, w.V, w.r)
+    rnd.run(dev, SEED, 0)
+    assert torch.equal(rnd.d, dev["base"])
+    dev2 = dict(dev, W=torch.zeros_like(dev["W"]), bias_scale=None)
+    rnd2 = SpecRound(w.B, w.K, w.V, w.r)
+    rnd2.run(dev2, SEED, 0)
+    assert torch.equal(rnd2.d, rnd.d) and torch.equal(rnd2.x, rnd.x)
+
+
+def test_status_bad_inputs(cuda_ok):
+    w = _small(B=8)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    rnd = SpecRound(w.B, w.K, w.V, w.r)
+    # last committed token out of range
+    bad = dict(dev, last_tok=dev["last_tok"].clone())
+    bad["last_tok"][3] = w.V + 5
+    rnd.run(bad, SEED, 0)
+    code, first = rnd.status()
+    assert code & bn.STATUS_BAD_TOKEN and first == 3
+    # NaN in a target row of request 5 (row 0 is always read)
+    bad = dict(dev, target=dev["target"].clone())
+    bad["target"][5, 0, 17] = float("nan")
+    rnd.run(bad, SEED, 0)
+    code, first = rnd.status()
+    assert code & bn.STATUS_BAD_ROW and first == 5
+    assert rnd.n_emit[5].item() >= 1
+    # negative temperature
+    bad = dict(dev, temp=dev["temp"].clone())
+    bad["temp"][6] = -1.0
+    rnd.run(bad, SEED, 0)
+    code, first = rnd.status()
+    assert code & bn.STATUS_BAD_TEMP and first == 6
+    # cut out of range, straight into verify
+    rnd.run(dev, SEED, 0)
+    assert rnd.status() == (0, -1)
+    cut = rnd.cut.clone()
+    cut[2] = w.K + 3
+    bn.verify(dev["target"], rnd.d, rnd.x, rnd.q_tok, cut, dev["temp"], SEED, 0, rnd.accepted,
+              rnd.out, rnd.n_emit, rnd.ws)
+    code, first = rnd.status()
+    assert code & bn.STATUS_BAD_CUT and first == 2
+    # and a clean round afterwards reports nothing
+    rnd.run(dev, SEED, 0)
+    assert rnd.status() == (0, -1)
+
+
+def test_argument_errors(cuda_ok):
+    w = _small(B=4, V=1024)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    rnd = SpecRound(w.B, w.K, w.V, w.r)
+    # misaligned logits (2-byte offset view)
+    flat = torch.empty(w.B * w.K * w.V + 8, dtype=torch.bfloat16, device="cuda")
+    mis = flat[1:1 + w.B * w.K * w.V].view(w.B, w.K, w.V)
+    with pytest.raises(bn.DSparkError, match="invalid argument"):
+        bn.draft_sample(mis, dev["U"], dev["W"], None, dev["last_tok"], dev["temp"], SEED, 0,
+                        rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws)
+    # workspace too small
+    with pytest.raises(bn.DSparkError, match="workspace"):
+        bn.draft_sample(dev["base"], dev["U"], dev["W"], None, dev["last_tok"], dev["temp"], SEED,
+                        0, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws[:64])
+    # V not a multiple of 8
+    t = torch.zeros(w.B, w.K + 1, 1001, dtype=torch.bfloat16, device="cuda")
+    dd = torch.zeros(w.B, w.K, 1001, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(bn.DSparkError, match="invalid argument"):
+        bn.verify(t, dd, rnd.x, rnd.q_tok, None, dev["temp"], SEED, 0, rnd.accepted, rnd.out,
+                  rnd.n_emit, rnd.ws)
+    # schedule larger than one CTA handles
+    big = torch.zeros(4096, 4, device="cuda")
+    with pytest.raises(bn.DSparkError, match="unsupported"):
+        bn.prefix_schedule(big, torch.ones(4, device="cuda"), torch.ones(4096 * 5, device="cuda"),
+                           0.0, bn.CUT_COST, 0.0, torch.empty(4096, dtype=torch.int32, device="cuda"),
+                           torch.empty(4096, 4, device="cuda"), rnd.ws)
+    assert rnd.status() == (0, -1)
+
+
+def test_round_replay_is_deterministic(cuda_ok):
+    w = _small(B=16)
+    inp = wl.generate(w)
+    rnd, dev = run_gpu(w, inp, 9)
+    out1 = rnd.out.clone()
+    rnd.run(dev, SEED, 9)
+    assert torch.equal(rnd.out, out1)
+    x1 = rnd.x.clone()
+    rnd.run(dev, SEED, 10)  # a new round id draws new uniforms
+    assert not torch.equal(rnd.x, x1)
