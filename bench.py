@@ -248,8 +248,9 @@ def main():
             step()
     torch.cuda.synchronize()
 
-    for _ in range(args.warmup):
-        graph.replay()
+    with torch.cuda.stream(stream):  # replay() launches on the current stream
+        for _ in range(args.warmup):
+            graph.replay()
     torch.cuda.synchronize()
     clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
     if clocks:
@@ -258,10 +259,11 @@ def main():
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        graph.replay()
-    e1.record(stream)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
     barrier(world)

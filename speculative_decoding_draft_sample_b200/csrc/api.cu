@@ -5,6 +5,7 @@
 
 #include "common.cuh"
 #include "draft.cuh"
+#include "draft_tc.cuh"
 #include "schedule.cuh"
 #include "verify.cuh"
 
@@ -130,8 +131,9 @@ int dspark_draft_sample(const void* base, const void* U, const void* W, const fl
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   a.nchunk = nchunks(V);
   cudaStream_t s = (cudaStream_t)stream;
+  const bool tc = draft_tc_supported(a);
   for (int k = 1; k <= K; ++k) {
-    cudaError_t e = draft_logits_simt_launch(a, k, s);
+    cudaError_t e = tc ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
     if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
     if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   }

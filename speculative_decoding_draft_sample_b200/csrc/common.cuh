@@ -28,7 +28,7 @@ __device__ __forceinline__ void report(Status* st, unsigned int bits, int reques
 constexpr float kLog2e = 1.44269504088896340736f;
 
 // Bounded spin limit for every device-side wait (mbarrier polls).
-constexpr long long kSpinLimit = 1ll << 26;
+constexpr long long kSpinLimit = 1ll << 22;
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy

@@ -95,6 +95,34 @@ __device__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* 
   phase ^= 1u;
 }
 
+// 16 bytes of shared memory as floats (8 bf16 or 4 fp32), in index order.
+template <int DT>
+struct Vec16;
+template <>
+struct Vec16<DSPARK_BF16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const uint16_t* p, float* v) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+};
+template <>
+struct Vec16<DSPARK_F32> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float* v) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x;
+    v[1] = q.y;
+    v[2] = q.z;
+    v[3] = q.w;
+  }
+};
+
 template <int DT>
 struct VerifyCta {
   using E = Elem<DT>;
@@ -119,6 +147,30 @@ struct VerifyCta {
     }
     __syncthreads();
     parity ^= 1;
+  }
+
+  // f(i, value) over this thread's elements of `buf`, in index order, 16 B at a time
+  template <class F>
+  __device__ __forceinline__ void each(const T* buf, F f) const {
+    constexpr int N = Vec16<DT>::N;
+    for (int i = t0; i < t1; i += N) {
+      float v[N];
+      Vec16<DT>::load(buf + i, v);
+#pragma unroll
+      for (int j = 0; j < N; ++j) f(i + j, v[j]);
+    }
+  }
+  // f(i, t_value, d_value) over this thread's elements of two buffers
+  template <class F>
+  __device__ __forceinline__ void each2(const T* b1, const T* b2, F f) const {
+    constexpr int N = Vec16<DT>::N;
+    for (int i = t0; i < t1; i += N) {
+      float v1[N], v2[N];
+      Vec16<DT>::load(b1 + i, v1);
+      Vec16<DT>::load(b2 + i, v2);
+#pragma unroll
+      for (int j = 0; j < N; ++j) f(i + j, v1[j], v2[j]);
+    }
   }
 
   // block max of v (all threads get it)
@@ -252,7 +304,15 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   const int b = blockIdx.x / c.C;
   c.lo = c.rank * a.slice;
   c.n = max(0, min(a.slice, a.V - c.lo));
-  c.per = ((c.n + kVThreads - 1) / kVThreads + 7) & ~7;
+  {
+    // each thread: a contiguous run of an odd number of 16-byte chunks, so that
+    // the 16-byte shared-memory loads of a quarter warp fall in distinct banks
+    constexpr int v16 = Vec16<DT>::N;
+    int per = (c.n + kVThreads - 1) / kVThreads;
+    per = (per + v16 - 1) / v16 * v16;
+    if (((per / v16) & 1) == 0) per += v16;
+    c.per = per;
+  }
   c.t0 = min(c.tid * c.per, c.n);
   c.t1 = min(c.t0 + c.per, c.n);
   T* tb = reinterpret_cast<T*>(dsm);
@@ -298,11 +358,10 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
       float mv = -INFINITY;
       int mi = 0x7fffffff;
       int bad = 0;
-      for (int i = c.t0; i < c.t1; ++i) {
-        const float v = E::to_float(tb[i]);
+      c.each(tb, [&](int i, float v) {
         bad |= bad_logit(v);
         argmax_merge(mv, mi, v, c.lo + i);
-      }
+      });
       warp_argmax(mv, mi);
       if (c.lane == 0) {
         red[c.warp] = mv;
@@ -337,11 +396,10 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     // pass A: max (scaled), bad flag, and t[x] of the draft being tested
     float mv = -INFINITY;
     int bad = 0;
-    for (int i = c.t0; i < c.t1; ++i) {
-      const float v = E::to_float(tb[i]);
+    c.each(tb, [&](int, float v) {
       bad |= bad_logit(v);
       mv = fmaxf(mv, v);
-    }
+    });
     mv = c.block_max(mv) * cs;
     bad = c.block_any(bad);
     float tx = -INFINITY;
@@ -357,7 +415,7 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     }
     // pass B: per-thread sums of exp2(z - M) in index order, block scan
     float s = 0.f;
-    for (int i = c.t0; i < c.t1; ++i) s += exp2f(E::to_float(tb[i]) * cs - M);
+    c.each(tb, [&](int, float v) { s += exp2f(v * cs - M); });
     const float tot = c.block_scan_store(s);
     c.gather(Exch{0.f, tot, 0.f, 0});
     Z = 0.f;
@@ -390,24 +448,25 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     // and draft row acc (q = softmax(d / temp), normaliser recomputed here)
     bulk_load(db, drow0 + (long long)acc * V + c.lo, nbytes, &bar, phase, st, b);
     float mq = -INFINITY;
-    for (int i = c.t0; i < c.t1; ++i) mq = fmaxf(mq, E::to_float(db[i]));
+    c.each(db, [&](int, float v) { mq = fmaxf(mq, v); });
     mq = c.block_max(mq) * cs;
     c.gather(Exch{mq, 0.f, 0.f, 0});
     float Mq = -INFINITY;
     for (int r = 0; r < c.C; ++r) Mq = fmaxf(Mq, got[r].f0);
     float sq = 0.f;
-    for (int i = c.t0; i < c.t1; ++i) sq += exp2f(E::to_float(db[i]) * cs - Mq);
+    c.each(db, [&](int, float v) { sq += exp2f(v * cs - Mq); });
     const float totq = c.block_scan_store(sq);
     c.gather(Exch{0.f, totq, 0.f, 0});
     float Zq = 0.f;
     for (int r = 0; r < c.C; ++r) Zq += got[r].f1;
-    auto resid = [&](int i) {
-      const float p = exp2f(E::to_float(tb[i]) * cs - M) / Z;
-      const float q = exp2f(E::to_float(db[i]) * cs - Mq) / Zq;
+    auto resid_v = [&](float tv, float dv) {
+      const float p = exp2f(tv * cs - M) / Z;
+      const float q = exp2f(dv * cs - Mq) / Zq;
       return fmaxf(0.f, p - q);
     };
+    auto resid = [&](int i) { return resid_v(E::to_float(tb[i]), E::to_float(db[i])); };
     float sr = 0.f;
-    for (int i = c.t0; i < c.t1; ++i) sr += resid(i);
+    c.each2(tb, db, [&](int, float tv, float dv) { sr += resid_v(tv, dv); });
     const float totr = c.block_scan_store(sr);
     c.gather(Exch{0.f, totr, 0.f, 0});
     float R = 0.f;
@@ -418,7 +477,7 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     } else {
       // exact-zero residual (floating point only): draw from p instead
       float s = 0.f;
-      for (int i = c.t0; i < c.t1; ++i) s += exp2f(E::to_float(tb[i]) * cs - M);
+      c.each(tb, [&](int, float v) { s += exp2f(v * cs - M); });
       c.block_scan_store(s);
       if (tid < c.C) got[tid] = rowtot[tid];
       __syncthreads();
