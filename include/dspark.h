@@ -74,6 +74,7 @@ enum { DSPARK_CUT_COST = 0, DSPARK_CUT_THRESHOLD = 1, DSPARK_CUT_NONE = 2 };
 #define DSPARK_STATUS_BAD_CUT 0x4u   /* cut outside [0, K]                       */
 #define DSPARK_STATUS_BAD_TEMP 0x8u  /* temperature negative or NaN             */
 #define DSPARK_STATUS_TIMEOUT 0x10u  /* a bounded device wait gave up           */
+#define DSPARK_STATUS_INTERNAL 0x20u /* a kernel precondition failed (alignment) */
 
 /*
  * Workspace bytes needed by operation `op` (DSPARK_OP_*) for these sizes

@@ -132,7 +132,9 @@ def draft_logits(base_k: np.ndarray, bias: np.ndarray, dtype: str,
         win = BF16_MID_WINDOW * np.abs(v)
     else:
         win = 2.0 ** -22 * np.abs(v) + r * 2.0 ** -23 * bias_abs
-    return out, np.abs(v - mid) <= win
+    with np.errstate(invalid="ignore"):  # infinite logits are never near a midpoint
+        flag = np.isfinite(v) & (np.abs(v - mid) <= win)
+    return out, flag
 
 
 def inverse_cdf(w: np.ndarray, u: np.ndarray, window: float = U_WINDOW, normalized: bool = True):

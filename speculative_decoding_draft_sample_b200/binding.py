@@ -21,6 +21,7 @@ F32, BF16 = 0, 1
 OP_DRAFT, OP_SCHEDULE, OP_VERIFY = 0, 1, 2
 CUT_COST, CUT_THRESHOLD, CUT_NONE = 0, 1, 2
 STATUS_BAD_TOKEN, STATUS_BAD_ROW, STATUS_BAD_CUT, STATUS_BAD_TEMP, STATUS_TIMEOUT = 1, 2, 4, 8, 16
+STATUS_INTERNAL = 32
 
 _lib = None
 

@@ -13,8 +13,26 @@ namespace dspark {
 struct Status {
   unsigned int code;       // OR of DSPARK_STATUS_* bits
   int first_bad_enc;       // INT_MAX - lowest offending request; 0 when none
-  unsigned int pad[62];
+  unsigned int where;      // first wait site that gave up (kWhere*), 0 when none
+  unsigned int pad[61];
 };
+
+// Wait sites recorded in Status::where when a bounded wait gives up.
+enum WaitSite : unsigned int {
+  kWhereVerifyLoad = 1,
+  kWhereTcWFull = 10,
+  kWhereTcWEmpty = 11,
+  kWhereTcBaseFull = 12,
+  kWhereTcBaseEmpty = 13,
+  kWhereTcAccFull = 14,
+  kWhereTcAccEmpty = 15,
+};
+
+__device__ __forceinline__ void report_wait(Status* st, unsigned int site, int request) {
+  atomicCAS(&st->where, 0u, site);
+  atomicOr(&st->code, (unsigned int)DSPARK_STATUS_TIMEOUT);
+  atomicMax(&st->first_bad_enc, 0x7fffffff - request);
+}
 static_assert(sizeof(Status) == 256, "status block is 256 bytes");
 constexpr size_t kStatusBytes = 256;
 
@@ -27,8 +45,34 @@ __device__ __forceinline__ void report(Status* st, unsigned int bits, int reques
 // so that exp2 gives the unnormalised softmax weight.
 constexpr float kLog2e = 1.44269504088896340736f;
 
-// Bounded spin limit for every device-side wait (mbarrier polls).
-constexpr long long kSpinLimit = 1ll << 22;
+// Bound on every device-side wait (mbarrier polls), in nanoseconds of the
+// global timer: a legitimate wait lasts microseconds, so a wait that passes
+// this limit reports DSPARK_STATUS_TIMEOUT instead of hanging the GPU.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for completion of the phase of parity `par` of the mbarrier at
+// shared address `bar`; false when it gave up. Each thread polls on its own;
+// callers reconverge the warp (__syncwarp) before any warp-aligned instruction.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t par) {
+  unsigned long long start = 0;
+  for (unsigned it = 0;; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+        : "=r"(ok)
+        : "r"(bar), "r"(par)
+        : "memory");
+    if (ok) return true;
+    if (it == 0) start = global_ns();
+    else if ((it & 255u) == 0 && global_ns() - start > kWaitLimitNs) return false;
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
@@ -97,6 +141,20 @@ struct Elem<DSPARK_BF16> {
   }
   __device__ __forceinline__ static float to_float(T v) { return bf16_bits_to_float(v); }
 };
+
+// 2^x on the special-function unit (ex2.approx; subnormal results flush to
+// zero, far below anything a sampling decision can see).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// max that propagates NaN (any NaN operand gives NaN)
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
 
 // A row is unusable for sampling when it holds NaN or +inf, or is all -inf.
 __device__ __forceinline__ bool bad_logit(float v) { return v != v || v == __int_as_float(0x7f800000); }

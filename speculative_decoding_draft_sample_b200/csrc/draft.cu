@@ -136,7 +136,7 @@ __global__ void __launch_bounds__(256) draft_logits_simt(DraftArgs a, int k) {
     const int b = b0 + bb;
     const float tau = (b < a.B) ? a.temp[b] : 1.f;
     if (tau > 0.f) {
-      const float e = col_ok ? exp2f(z[bb] - cm[bb]) : 0.f;
+      const float e = (col_ok && cm[bb] != -INFINITY) ? ex2(z[bb] - cm[bb]) : 0.f;
       const float s = warp_sum(e);
       if (lane == 0) red_s[warp][bb] = s;
     }
@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
   __shared__ int s_chunk;
   __shared__ float s_rem;
   __shared__ int s_tok;
+  __shared__ int s_last;
 
   const int b = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
   for (int w = 1; w < 8; ++w) M = fmaxf(M, wmax[w]);
 
   float s = 0.f;
-  for (int c = c0; c < c1; ++c) s += P[c].y * exp2f(P[c].x - M);
+  for (int c = c0; c < c1; ++c) s += (P[c].x == -INFINITY) ? 0.f : P[c].y * ex2(P[c].x - M);
   const float incl_w = warp_inclusive_scan(s);
   if (lane == 31) wsum[warp] = incl_w;
   __syncthreads();
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
     float rem = thr - excl;
     int found = -1, lastpos = -1;
     for (int c = c0; c < c1; ++c) {
-      const float vc = P[c].y * exp2f(P[c].x - M);
+      const float vc = (P[c].x == -INFINITY) ? 0.f : P[c].y * ex2(P[c].x - M);
       if (vc > 0.f) lastpos = c;
       if (rem < vc) {
         found = c;
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
     // rounding: u*Z at or past the total; take the last positive element
     int lastpos = -1;
     for (int c = nch - 1; c >= 0; --c)
-      if (P[c].y * exp2f(P[c].x - M) > 0.f) {
+      if (P[c].x != -INFINITY && P[c].y * ex2(P[c].x - M) > 0.f) {
         lastpos = c;
         break;
       }
@@ -300,7 +301,7 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
   const T* d = static_cast<const T*>(a.d);
   float w = 0.f;
   if (ch >= 0 && tid < kChunk && vi < a.V)
-    w = exp2f(E::load(d, ((long long)b * a.K + (k - 1)) * a.V + vi) * c - M);
+    w = ex2(fmaf(E::load(d, ((long long)b * a.K + (k - 1)) * a.V + vi), c, -M));
   const float iw = warp_inclusive_scan(w);
   __syncthreads();
   if (lane == 31) wsum[warp] = iw;
@@ -313,12 +314,13 @@ __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
   __syncthreads();
   int tok = s_tok;
   if (tok == 0x7fffffff) {
-    // rounding fallback: last positive element of the chunk
-    if (tid == 0) s_tok = -1;
+    // rounding fallback: last positive element of the chunk (a second
+    // variable: other threads may still be reading s_tok)
+    if (tid == 0) s_last = -1;
     __syncthreads();
-    if (w > 0.f) atomicMax(&s_tok, tid);
+    if (w > 0.f) atomicMax(&s_last, tid);
     __syncthreads();
-    tok = s_tok;
+    tok = s_last;
   }
   if (tid == (tok < 0 ? 0 : tok)) {
     const int xi = (tok < 0) ? 0 : ch * kChunk + tok;

@@ -17,9 +17,12 @@
 //   warp 0     TMA producer of W tiles (4-stage-per-tile ring of 32 KB stages)
 //   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer
 //   warp 2     TMA producer of base tiles (ring of 16 KB [128 x 64] blocks)
-//   warps 4-7  epilogue: tcgen05.ld of the accumulator (lane = request row),
-//              + base, round to bf16, write d back into the staged block, TMA
-//              store of d, running (max, sum) per row.
+//   warps 4-11 epilogue, two halves of four warps (one per TMEM lane
+//              quadrant): half h takes column blocks h and h+2 of every tile.
+//              tcgen05.ld of the accumulator (lane = request row), + base,
+//              round to bf16 (packed), write d back into the staged block, TMA
+//              store of d, running (max, sum exp2) per row; the halves merge
+//              their row statistics through shared memory at the end of a tile.
 // Every wait on an mbarrier is bounded; a CTA that gives up reports
 // DSPARK_STATUS_TIMEOUT and winds down instead of hanging.
 #include <cuda.h>
@@ -31,12 +34,12 @@ namespace dspark {
 
 namespace tc {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;      // 4 role warps + 8 epilogue warps
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
 constexpr int kWStages = 3;         // W ring depth (stages of 64 k-rows x 256 vocab)
 constexpr int kWStageBytes = 64 * 256 * 2;
-constexpr int kBaseSlots = 4;       // base/d ring depth ([128 x 64] blocks)
+constexpr int kBaseSlots = 4;       // base/d blocks of one tile ([128 x 64] each)
 constexpr int kBlockBytes = 128 * 64 * 2;
 constexpr int kABytes = 128 * 256 * 2;  // gathered U rows, 4 k-blocks of [128 x 64]
 
@@ -46,7 +49,9 @@ constexpr int kOffW = kOffA + kABytes;
 constexpr int kOffBase = kOffW + kWStages * kWStageBytes;
 constexpr int kOffBar = kOffBase + kBaseSlots * kBlockBytes;
 constexpr int kNumBars = 2 * kWStages + 2 * kBaseSlots + 4;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;  // + tmem slot + alignment slack
+constexpr int kOffX = kOffBar + kNumBars * 8 + 16;              // [2][128] float2 row stats
+constexpr int kSmemBytes = kOffX + 2 * 128 * 8;
+static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
 
 // instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 MN-major,
 // M = 128, N = 256
@@ -78,19 +83,8 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
 }
-// Bounded wait for the phase of parity `par`; false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t par) {
-  const uint32_t a = su32(b);
-  for (long long it = 0; it < kSpinLimit; ++it) {
-    uint32_t ok;
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(ok)
-        : "r"(a), "r"(par)
-        : "memory");
-    if (ok) return true;
-  }
-  return false;
+  return mbar_wait_bounded(su32(b), par);
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
@@ -120,16 +114,26 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Named barrier of the four epilogue warps that also ORs a flag across them,
-// so that giving up after a timed-out wait is one decision for all 128 threads.
+// Named barrier of the eight epilogue warps that also ORs a flag across them,
+// so that giving up after a timed-out wait is one decision for all 256 threads.
 __device__ __forceinline__ bool epi_bar_any(bool flag) {
   uint32_t r;
   asm volatile(
-      "{ .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+      "{ .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 3, 256, p;\n selp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
       : "r"((uint32_t)flag)
       : "memory");
   return r != 0;
+}
+
+// Two fp32 values rounded to nearest-even bf16, packed (lo in the low half).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ void half_bar(int h) {  // the four warps of one epilogue half
+  asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
@@ -168,8 +172,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     draft_logits_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_base,
                     const __grid_constant__ CUtensorMap map_d, Params p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 128-byte-swizzled TMA tiles and MMA operands need 1024-byte alignment
+  if (su32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) report(p.status, DSPARK_STATUS_INTERNAL, 0);
+    return;
+  }
+  unsigned char* smem = smem_raw;
   unsigned char* sA = smem + kOffA;
   unsigned char* sW = smem + kOffW;
   unsigned char* sBase = smem + kOffBase;
@@ -182,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* t_empty = t_full + 2;            // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+  float2* xstat = reinterpret_cast<float2*>(smem + kOffX);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int mt_local = blockIdx.x % p.m_per_launch;
@@ -204,7 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&t_full[i], 1);
-      mbar_init(&t_empty[i], 128);
+      mbar_init(&t_empty[i], 256);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -252,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % kWStages;
         if (*(volatile int*)abort_flag || !mbar_wait(&w_empty[s], ((it / kWStages) & 1) ^ 1)) {
+          if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcWEmpty, m0);
           *(volatile int*)abort_flag = 1;
           stop = true;
           break;
@@ -269,28 +279,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[q] >= 0) mbar_wait(&w_full[q], (last[q] / kWStages) & 1);
   } else if (warp == 2 && lane == 0) {
     // ---------------- base producer ----------------
-    int g = 0;
-    int last[kBaseSlots];
-    for (int q = 0; q < kBaseSlots; ++q) last[q] = -1;
+    // block j of every tile goes to ring slot j; the phase is the tile parity
+    int last_tile = -1;
     for (int i = 0; i < n_my; ++i) {
       const int n0 = (nt0 + i * nstride) * kTileN;
       bool stop = false;
-      for (int j = 0; j < 4; ++j, ++g) {
-        const int s = g % kBaseSlots;
-        if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[s], ((g / kBaseSlots) & 1) ^ 1)) {
+      for (int j = 0; j < 4; ++j) {
+        if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[j], (i & 1) ^ 1)) {
+          if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcBaseEmpty, m0);
           *(volatile int*)abort_flag = 1;
           stop = true;
           break;
         }
-        mbar_expect_tx(&b_full[s], kBlockBytes);
-        tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + j * 64, p.k - 1, m0, &b_full[s]);
-        last[s] = g;
+        mbar_expect_tx(&b_full[j], kBlockBytes);
+        tma_load_3d(sBase + j * kBlockBytes, &map_base, n0 + j * 64, p.k - 1, m0, &b_full[j]);
       }
+      last_tile = i;
       if (stop) break;
     }
-    if (*(volatile int*)abort_flag)
-      for (int q = 0; q < kBaseSlots; ++q)
-        if (last[q] >= 0) mbar_wait(&b_full[q], (last[q] / kBaseSlots) & 1);
+    if (*(volatile int*)abort_flag && last_tile >= 0)
+      for (int j = 0; j < 4; ++j) mbar_wait(&b_full[j], last_tile & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     int it = 0;
@@ -299,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < n_my; ++i) {
       const int buf = i & 1;
       if (*(volatile int*)abort_flag || !mbar_wait(&t_empty[buf], ((i >> 1) & 1) ^ 1)) {
+        if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcAccEmpty, m0);
         *(volatile int*)abort_flag = 1;
         break;
       }
@@ -308,6 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % kWStages;
         if (!mbar_wait(&w_full[s], (it / kWStages) & 1)) {
+          report_wait(p.status, kWhereTcWFull, m0);
           ok = false;
           break;
         }
@@ -350,6 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     // ---------------- epilogue ----------------
     const int q = warp & 3;             // TMEM lane quadrant
+    const int h = (warp - 4) >> 2;      // half: column blocks h and h + 2
     const int row = q * 32 + lane;      // request row inside the tile
     const int b = m0 + row;
     const bool valid = b < p.B;
@@ -358,112 +369,141 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float cs = greedy ? 1.f : kLog2e / tau;
     const float sc = (valid && p.bias_scale) ? p.bias_scale[b] : 1.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
-    int g = 0;
-    bool fail = false;
-    for (int i = 0; i < n_my && !fail; ++i) {
+    const bool elected = (warp == 4 + 4 * h) && lane == 0;
+    bool miss = false;
+    for (int i = 0; i < n_my; ++i) {
       const int nt = nt0 + i * nstride;
       const int n0 = nt * kTileN;
       const int buf = i & 1;
-      bool miss = !mbar_wait(&t_full[buf], (i >> 1) & 1);
+      if (!mbar_wait(&t_full[buf], (i >> 1) & 1)) {
+        miss = true;
+        report_wait(p.status, kWhereTcAccFull, m0);
+      }
+      __syncwarp();
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      float run_m = -INFINITY, run_s = 0.f;
+      // sampled rows: running max of z = d * cs and sum of 2^(z - max)
+      // greedy rows: running (max d, argmax), NaN-propagating check value
+      float run_m = -INFINITY, run_s = 0.f, chk = -INFINITY;
       int arg = 0x7fffffff;
-      bool bad = false;
-      for (int j = 0; j < 4; ++j, ++g) {
-        const int s = g % kBaseSlots;
-        miss |= !mbar_wait(&b_full[s], (g / kBaseSlots) & 1);
+#pragma unroll 1
+      for (int jj = 0; jj < 2; ++jj) {
+        const int j = h + 2 * jj;       // column block, also its ring slot
+        if (!mbar_wait(&b_full[j], i & 1)) {
+          miss = true;
+          report_wait(p.status, kWhereTcBaseFull, m0);
+        }
+        __syncwarp();  // tcgen05.ld is warp-aligned: every lane, together
         float acc[64];
         const uint32_t col = tmem + lane_base + buf * kTileN + j * 64;
         tmem_ld32(col, acc);
         tmem_ld32(col + 32, acc + 32);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        unsigned char* blk = sBase + s * kBlockBytes + row * 128;
-        float z[64];
+        unsigned char* blk = sBase + j * kBlockBytes + row * 128;
+        uint32_t dp[32];                // the block's 64 stored logits, packed
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4* ptr = reinterpret_cast<uint4*>(blk + ((c ^ (row & 7)) << 4));
-          uint4 v = *ptr;
-          uint32_t w[4] = {v.x, v.y, v.z, v.w};
+          const uint4 v = *ptr;
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float b0 = __uint_as_float(w[h] << 16);
-            const float b1 = __uint_as_float(w[h] & 0xffff0000u);
-            const uint16_t d0 = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(sc, acc[c * 8 + 2 * h], b0)));
-            const uint16_t d1 = __bfloat16_as_ushort(__float2bfloat16_rn(fmaf(sc, acc[c * 8 + 2 * h + 1], b1)));
-            w[h] = (uint32_t)d0 | ((uint32_t)d1 << 16);
-            z[c * 8 + 2 * h] = __uint_as_float((uint32_t)d0 << 16);
-            z[c * 8 + 2 * h + 1] = __uint_as_float((uint32_t)d1 << 16);
+          for (int e = 0; e < 4; ++e) {
+            const float y0 = fmaf(sc, acc[c * 8 + 2 * e], __uint_as_float(w[e] << 16));
+            const float y1 = fmaf(sc, acc[c * 8 + 2 * e + 1], __uint_as_float(w[e] & 0xffff0000u));
+            dp[c * 4 + e] = pack_bf16x2(y0, y1);
           }
-          *ptr = make_uint4(w[0], w[1], w[2], w[3]);
+          *ptr = make_uint4(dp[c * 4], dp[c * 4 + 1], dp[c * 4 + 2], dp[c * 4 + 3]);
         }
-        // statistics over the valid columns of this block
         const int vcols = min(64, p.V - (n0 + j * 64));
-        if (valid) {
+        if (valid && vcols > 0) {
           if (greedy) {
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-              if (e < vcols) {
-                bad |= bad_logit(z[e]);
-                argmax_merge(run_m, arg, z[e], n0 + j * 64 + e);
+              const float dv = __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16));
+              if (vcols == 64 || e < vcols) {
+                chk = max_nan(chk, dv);
+                if (dv > run_m) {
+                  run_m = dv;
+                  arg = n0 + j * 64 + e;
+                }
               }
             }
           } else {
             float bm = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 64; ++e) {
-              if (e < vcols) {
-                bad |= bad_logit(z[e]);
-                z[e] *= cs;
-                bm = fmaxf(bm, z[e]);
-              }
+              const float dv = __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16));
+              if (vcols == 64 || e < vcols) bm = max_nan(bm, dv);
             }
-            const float nm = fmaxf(run_m, bm);
-            float acc_s = 0.f;
+            if (bm != bm) {
+              run_s = NAN;  // a NaN logit: the chunk partial reports it
+            } else {
+              const float nm = fmaxf(run_m, bm * cs);
+              if (nm != -INFINITY) {  // -inf entries weigh nothing; +inf makes the sum NaN
+                const float neg = -nm;
+                float acc_s = 0.f;
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              if (e < vcols) acc_s += exp2f(z[e] - nm);
-            run_s = (run_m == -INFINITY ? 0.f : run_s * exp2f(run_m - nm)) + acc_s;
-            run_m = nm;
+                for (int e = 0; e < 64; ++e) {
+                  const float dv = __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16));
+                  if (vcols == 64 || e < vcols) acc_s += ex2(fmaf(dv, cs, neg));
+                }
+                run_s = (run_m == -INFINITY ? 0.f : run_s * ex2(run_m - nm)) + acc_s;
+              }
+              run_m = nm;
+            }
           }
         }
         fence_async_smem();
-        if (epi_bar_any(miss)) {  // a wait gave up somewhere: every epilogue thread stops here
-          fail = true;
-          *(volatile int*)abort_flag = 1;
-          break;
-        }
-        if (warp == 4 && lane == 0) {
-          tma_store_3d(&map_d, sBase + s * kBlockBytes, n0 + j * 64, p.k - 1, m0);
+        __syncwarp();
+        half_bar(h);
+        if (elected) {
+          tma_store_3d(&map_d, sBase + j * kBlockBytes, n0 + j * 64, p.k - 1, m0);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          // the previous block's smem has been read by its store: free that slot
-          asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-          if (g > 0) mbar_arrive(&b_empty[(g - 1) % kBaseSlots]);
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          mbar_arrive(&b_empty[j]);
         }
+        __syncwarp();  // lane 0 may still be in the store above
       }
-      if (fail) break;
       // this thread is done reading accumulator buffer `buf`
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&t_empty[buf]);
-      if (valid) {
+      // merge the two halves' statistics of this row
+      float2* xs = xstat + (i & 1) * 128;
+      if (h == 1) {
+        // greedy rows fold the NaN / +inf check into the max
+        const bool bad_g = greedy && (chk != chk || chk == INFINITY);
+        xs[row] = greedy ? make_float2(bad_g ? NAN : run_m, __int_as_float(arg))
+                         : make_float2(run_m, run_s);
+      }
+      __syncwarp();
+      if (epi_bar_any(miss)) {  // a wait gave up somewhere: every epilogue thread stops here
+        *(volatile int*)abort_flag = 1;
+        break;
+      }
+      if (h == 0 && valid) {
+        const float2 o = xs[row];
         float2 part;
         if (greedy) {
-          part.x = bad ? NAN : run_m;
-          part.y = __int_as_float(arg);
+          float m = run_m;
+          int a = arg;
+          argmax_merge(m, a, o.x, __float_as_int(o.y));
+          const bool bad = chk != chk || chk == INFINITY || o.x != o.x;
+          part.x = bad ? NAN : m;
+          part.y = __int_as_float(a);
         } else {
-          part.x = run_m;
-          part.y = bad ? NAN : run_s;
+          const float m = fmaxf(run_m, o.x);
+          const float s0 = run_m == -INFINITY ? 0.f : run_s * ex2(run_m - m);
+          const float s1 = o.x == -INFINITY ? 0.f : o.y * ex2(o.x - m);
+          part.x = m;
+          part.y = s0 + s1;  // NaN propagates; a chunk all at -inf is (-inf, 0)
         }
         p.partials[(long long)b * p.nchunk + nt] = part;
       }
     }
-    if (warp == 4 && lane == 0) {
-      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-      if (g > 0 && !fail) mbar_arrive(&b_empty[(g - 1) % kBaseSlots]);
-    }
+    if (elected) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
+  __syncwarp();  // role lanes rejoin their warps before the block barrier
   __syncthreads();
-  if (tid == 0 && *(volatile int*)abort_flag) report(p.status, DSPARK_STATUS_TIMEOUT, m0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (warp == 1) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");

@@ -47,7 +47,9 @@ __device__ __forceinline__ int cluster_size() {
   return (int)r;
 }
 // All threads of all CTAs of the cluster; release/acquire orders shared memory.
+// The barrier instructions are warp-aligned, so the warp reconverges first.
 __device__ __forceinline__ void cluster_sync() {
+  __syncwarp();
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 // Reads 16 bytes at the same shared-memory offset in CTA `rank` of the cluster.
@@ -65,7 +67,11 @@ __device__ __forceinline__ uint4 dsmem_load16(const void* local, int rank) {
 // Bulk copy of `bytes` (multiple of 16) from global to this CTA's shared memory,
 // completing on `bar`; every thread then waits (bounded) for phase `phase`.
 __device__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                          uint32_t& phase, Status* st, int request) {
+                          uint32_t& phase, Status* st, int request, int* dead) {
+  if (*(volatile int*)dead) {  // this CTA already gave up once: no more copies or waits
+    phase ^= 1u;
+    return;
+  }
   const uint32_t b = smem_u32(bar);
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
@@ -79,19 +85,13 @@ __device__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* 
           : "memory");
     }
   }
-  uint32_t done = 0;
-  long long it = 0;
-  while (!done) {
-    asm volatile(
-        "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-        : "=r"(done)
-        : "r"(b), "r"(phase)
-        : "memory");
-    if (!done && ++it > kSpinLimit) {
-      if (threadIdx.x == 0) report(st, DSPARK_STATUS_TIMEOUT, request);
-      break;
-    }
+  if (!mbar_wait_bounded(b, phase)) {
+    if (threadIdx.x == 0) report_wait(st, kWhereVerifyLoad, request);
+    mbar_wait_bounded(b, phase);  // give an in-flight copy a last chance to land
+    *(volatile int*)dead = 1;
   }
+  __syncwarp();
+  __syncthreads();  // every thread sees the same `dead` before the next copy
   phase ^= 1u;
 }
 
@@ -131,13 +131,16 @@ struct VerifyCta {
   int C, rank, tid, lane, warp;
   int lo, n, per, t0, t1;  // slice [lo, lo+n); this thread's elements [t0, t1) of it
   Exch* ex;                // [2] published slots (double buffered)
-  Exch* got;               // [kMaxCluster] gathered copies
-  float* part;             // [kVThreads] per-thread partial sums
-  float* excl;             // [kVThreads] their exclusive block scan
+  Exch* got;               // [kMaxCluster] gathered copies (read-only after a gather)
+  float* rw;               // [kMaxCluster] per-rank weights of the placement at hand
+  float* pm;               // [kVThreads] per-thread running max (online rows)
+  float* ps;               // [kVThreads] per-thread sums
+  float* excl;             // [kVThreads] exclusive block scan of the weights
   float* red;              // [32] scratch
   int* sint;               // [4] scratch
   int parity;
 
+  // Publishes this CTA's value and gathers every CTA's (one cluster barrier).
   __device__ void gather(const Exch& mine) {
     if (tid == 0) ex[parity] = mine;
     cluster_sync();
@@ -160,7 +163,6 @@ struct VerifyCta {
       for (int j = 0; j < N; ++j) f(i + j, v[j]);
     }
   }
-  // f(i, t_value, d_value) over this thread's elements of two buffers
   template <class F>
   __device__ __forceinline__ void each2(const T* b1, const T* b2, F f) const {
     constexpr int N = Vec16<DT>::N;
@@ -173,62 +175,95 @@ struct VerifyCta {
     }
   }
 
-  // block max of v (all threads get it)
-  __device__ float block_max(float v) {
-    v = warp_max(v);
-    if (lane == 0) red[warp] = v;
-    __syncthreads();
-    float m = red[0];
-    for (int w = 1; w < kVThreads / 32; ++w) m = fmaxf(m, red[w]);
-    __syncthreads();
-    return m;
-  }
-  __device__ int block_any(int v) {
-    v = __any_sync(0xffffffffu, v);
-    if (lane == 0) sint[0] = 0;
-    __syncthreads();
-    if (v && lane == 0) atomicOr(&sint[0], 1);
-    __syncthreads();
-    const int r = sint[0];
-    __syncthreads();
-    return r;
-  }
-  // stores part[tid] = s and excl[tid] = exclusive scan; returns the block total
-  __device__ float block_scan_store(float s) {
-    const float incl = warp_inclusive_scan(s);
-    if (lane == 31) red[warp] = incl;
-    __syncthreads();
-    float pre = 0.f, tot = 0.f;
-    for (int w = 0; w < kVThreads / 32; ++w) {
-      if (w < warp) pre += red[w];
-      tot += red[w];
+  // Online (max, sum 2^(z - max)) of z = v * cs over this thread's elements,
+  // kept in pm/ps for a later placement; returns the CTA's pair (thread 0's
+  // result is the one published). NaN or +inf anywhere makes the sum NaN.
+  __device__ float2 online_stats(const T* buf, float cs) {
+    constexpr int N = Vec16<DT>::N;
+    float m = -INFINITY, sum = 0.f;
+    for (int i = t0; i < t1; i += N) {
+      float v[N];
+      Vec16<DT>::load(buf + i, v);
+      float vm = v[0];
+#pragma unroll
+      for (int j = 1; j < N; ++j) vm = max_nan(vm, v[j]);
+      const float zm = vm * cs;
+      if (zm != zm) {  // NaN in this vector
+        sum = NAN;
+        continue;
+      }
+      if (zm > m) {
+        sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
+        m = zm;
+      }
+      if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
+        const float neg = -m;
+#pragma unroll
+        for (int j = 0; j < N; ++j) sum += ex2(fmaf(v[j], cs, neg));
+      }
     }
-    part[tid] = s;
-    excl[tid] = pre + incl - s;
+    pm[tid] = m;
+    ps[tid] = sum;
+    // warp combine, then the 8 warp results
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+      const float mm = fmaxf(m, m2);
+      const float a = (m == -INFINITY) ? 0.f : sum * ex2(m - mm);
+      const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2(m2 - mm);
+      sum = (sum != sum || s2 != s2) ? NAN : a + b;
+      m = mm;
+    }
+    if (lane == 0) {
+      red[warp] = m;
+      red[8 + warp] = sum;
+    }
     __syncthreads();
-    return tot;
+    float M = red[0], S = red[8];
+    for (int w = 1; w < kVThreads / 32; ++w) {
+      const float mm = fmaxf(M, red[w]);
+      const float a = (M == -INFINITY) ? 0.f : S * ex2(M - mm);
+      const float b = (red[w] == -INFINITY) ? 0.f : red[8 + w] * ex2(red[w] - mm);
+      S = (S != S || red[8 + w] != red[8 + w]) ? NAN : a + b;
+      M = mm;
+    }
+    __syncthreads();
+    return make_float2(M, S);
   }
 
-  // Inverse-CDF placement of `thr` on weights wfun(i) (slice-local index i)
-  // whose per-rank totals are got[r].f1 (rank prefix computed here). Returns
-  // the global token index in every thread of the owning CTA, -1 in the other
-  // CTAs, and -2 everywhere if no rank holds positive mass. Control flow is
-  // uniform inside the CTA; no cluster exchange happens here.
+  // Block sum of per-thread values (also kept in ps for a later placement).
+  __device__ float block_sum_keep(float v) {
+    ps[tid] = v;
+    pm[tid] = 0.f;  // weights are ps * 2^(pm - 0)
+    const float w = warp_sum(v);
+    if (lane == 0) red[warp] = w;
+    __syncthreads();
+    float t = 0.f;
+    for (int i = 0; i < kVThreads / 32; ++i) t += red[i];
+    __syncthreads();
+    return t;
+  }
+
+  // Inverse-CDF placement of `thr` on weights wfun(i) (slice-local index i).
+  // Per-rank totals are rw[r]; this thread's total weight is
+  // ps[tid] * 2^(pm[tid] - Mref). Returns the global token index in every
+  // thread of the owning CTA, -1 in the other CTAs, and -2 everywhere if no
+  // rank holds positive mass. No cluster exchange happens here.
   template <class F>
-  __device__ int place(float thr, F wfun) {
-    // owner rank: first r with thr < P_r + s_r (positive s_r); else last positive
+  __device__ int place(float thr, float Mref, F wfun) {
     int owner = -1, lastpos = -1;
     float P = 0.f, Pown = 0.f;
     for (int r = 0; r < C; ++r) {
-      const float s = got[r].f1;
-      if (s > 0.f) {
+      const float sr = rw[r];
+      if (sr > 0.f) {
         lastpos = r;
-        if (owner < 0 && thr < P + s) {
+        if (owner < 0 && thr < P + sr) {
           owner = r;
           Pown = P;
         }
       }
-      P += s;
+      P += sr;
     }
     bool fallback = false;
     if (owner < 0) {
@@ -237,18 +272,25 @@ struct VerifyCta {
     }
     if (owner < 0) return -2;
     if (owner != rank) return -1;
-    float rem = fallback ? INFINITY : thr - Pown;
-    // owner thread: first t with rem < excl_t + part_t
+    // this thread's weight and its exclusive prefix in index order
+    const float wt = (pm[tid] == -INFINITY) ? 0.f : ps[tid] * ex2(pm[tid] - Mref);
+    const float incl = warp_inclusive_scan(wt);
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    float pre = 0.f;
+    for (int w = 0; w < warp; ++w) pre += red[w];
+    const float ex_t = pre + incl - wt;
+    const float rem = fallback ? INFINITY : thr - Pown;
     if (tid == 0) sint[1] = 0x7fffffff;
     __syncthreads();
-    if (part[tid] > 0.f && rem < excl[tid] + part[tid]) atomicMin(&sint[1], tid);
+    if (wt > 0.f && rem < ex_t + wt) atomicMin(&sint[1], tid);
     __syncthreads();
     int ot = sint[1];
     bool tfall = fallback;
     if (ot == 0x7fffffff) {  // rounding: last thread with positive mass
       if (tid == 0) sint[2] = -1;
       __syncthreads();
-      if (part[tid] > 0.f) atomicMax(&sint[2], tid);
+      if (wt > 0.f) atomicMax(&sint[2], tid);
       __syncthreads();
       ot = sint[2];
       tfall = true;
@@ -256,7 +298,7 @@ struct VerifyCta {
     if (tid == 0) sint[3] = -1;
     __syncthreads();
     if (tid == ot) {
-      float r2 = tfall ? INFINITY : rem - excl[tid];
+      float r2 = tfall ? INFINITY : rem - ex_t;
       int found = -1, lastp = -1;
       for (int i = t0; i < t1; ++i) {
         const float w = wfun(i);
@@ -277,6 +319,19 @@ struct VerifyCta {
   }
 };
 
+// Combined (max, sum) of the gathered per-CTA online pairs (f0, f1), in rank order.
+__device__ __forceinline__ float2 combine_ranks(const Exch* got, int C) {
+  float M = -INFINITY;
+  for (int r = 0; r < C; ++r) M = fmaxf(M, got[r].f0);
+  float Z = 0.f;
+  for (int r = 0; r < C; ++r) {
+    const float s = got[r].f1;
+    if (s != s) return make_float2(M, NAN);
+    Z += (got[r].f0 == -INFINITY) ? 0.f : s * ex2(got[r].f0 - M);
+  }
+  return make_float2(M, Z);
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   using E = Elem<DT>;
@@ -284,9 +339,11 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ Exch ex[2];
   __shared__ Exch got[kMaxCluster];
-  __shared__ float part[kVThreads], excl[kVThreads], red[32];
+  __shared__ float rw[kMaxCluster];
+  __shared__ float pm[kVThreads], ps[kVThreads], excl[kVThreads], red[32];
   __shared__ int sint[4];
   __shared__ __align__(8) uint64_t bar;
+  __shared__ int dead;
 
   VerifyCta<DT> c;
   c.C = cluster_size();
@@ -296,7 +353,9 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   c.warp = c.tid >> 5;
   c.ex = ex;
   c.got = got;
-  c.part = part;
+  c.rw = rw;
+  c.pm = pm;
+  c.ps = ps;
   c.excl = excl;
   c.red = red;
   c.sint = sint;
@@ -321,6 +380,7 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   const int tid = c.tid;
 
   if (tid == 0) {
+    dead = 0;
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar)) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -333,7 +393,7 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     if (tid == 0 && c.rank == 0) report(st, DSPARK_STATUS_BAD_CUT, b);
     L = L < 0 ? 0 : K;
   }
-  float tau = a.temp[b];
+  const float tau = a.temp[b];
   if (tau != tau || tau < 0.f) {
     if (tid == 0 && c.rank == 0) report(st, DSPARK_STATUS_BAD_TEMP, b);
   }
@@ -346,32 +406,40 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   int acc = 0;
   bool rejected = false;
   bool badrow = false;
-  float M = 0.f, Z = 0.f;     // current target row's max (scaled) and sum
+  float M = 0.f, Z = 0.f;  // current target row's max (z units) and sum
   int y = -1;
-  Exch rowtot[kMaxCluster];   // per-rank sums of the current target row
 
   for (int j = 0; j <= L; ++j) {
-    bulk_load(tb, target + (long long)j * V + c.lo, nbytes, &bar, phase, st, b);
+    bulk_load(tb, target + (long long)j * V + c.lo, nbytes, &bar, phase, st, b, &dead);
     const int xk = (j < L) ? a.x[(long long)b * K + j] : -1;
     if (j < L && (xk < 0 || xk >= V) && tid == 0 && c.rank == 0) report(st, DSPARK_STATUS_BAD_TOKEN, b);
     if (greedy) {
-      float mv = -INFINITY;
+      float mv = -INFINITY, chk = -INFINITY;
       int mi = 0x7fffffff;
-      int bad = 0;
       c.each(tb, [&](int i, float v) {
-        bad |= bad_logit(v);
-        argmax_merge(mv, mi, v, c.lo + i);
+        chk = max_nan(chk, v);
+        if (v > mv) {
+          mv = v;
+          mi = c.lo + i;
+        }
       });
       warp_argmax(mv, mi);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) chk = max_nan(chk, __shfl_xor_sync(0xffffffffu, chk, o));
       if (c.lane == 0) {
         red[c.warp] = mv;
+        red[8 + c.warp] = chk;
         reinterpret_cast<int*>(red)[16 + c.warp] = mi;
       }
-      bad = c.block_any(bad);
-      float m = red[0];
-      int mm = reinterpret_cast<int*>(red)[16];
-      for (int w = 1; w < kVThreads / 32; ++w) argmax_merge(m, mm, red[w], reinterpret_cast<int*>(red)[16 + w]);
       __syncthreads();
+      float m = red[0], ck = red[8];
+      int mm = reinterpret_cast<int*>(red)[16];
+      for (int w = 1; w < kVThreads / 32; ++w) {
+        argmax_merge(m, mm, red[w], reinterpret_cast<int*>(red)[16 + w]);
+        ck = max_nan(ck, red[8 + w]);
+      }
+      __syncthreads();
+      const bool bad = (ck != ck) || ck == INFINITY;
       c.gather(Exch{m, 0.f, 0.f, mm | (bad ? (int)0x80000000 : 0)});
       float gm = -INFINITY;
       int gi = 0x7fffffff;
@@ -393,37 +461,21 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
       continue;
     }
 
-    // pass A: max (scaled), bad flag, and t[x] of the draft being tested
-    float mv = -INFINITY;
-    int bad = 0;
-    c.each(tb, [&](int, float v) {
-      bad |= bad_logit(v);
-      mv = fmaxf(mv, v);
-    });
-    mv = c.block_max(mv) * cs;
-    bad = c.block_any(bad);
+    // one online pass: (max, sum) of z = t * cs, and t[x] of the draft tested
+    const float2 mz = c.online_stats(tb, cs);
     float tx = -INFINITY;
     if (xk >= c.lo && xk < c.lo + c.n) tx = E::to_float(tb[xk - c.lo]) * cs;
-    c.gather(Exch{mv, 0.f, tx, bad});
-    M = -INFINITY;
+    c.gather(Exch{mz.x, mz.y, tx, 0});
     float gtx = -INFINITY;
-    bool gbad = false;
-    for (int r = 0; r < c.C; ++r) {
-      M = fmaxf(M, got[r].f0);
-      gtx = fmaxf(gtx, got[r].f2);
-      gbad |= got[r].i0 != 0;
-    }
-    // pass B: per-thread sums of exp2(z - M) in index order, block scan
-    float s = 0.f;
-    c.each(tb, [&](int, float v) { s += exp2f(v * cs - M); });
-    const float tot = c.block_scan_store(s);
-    c.gather(Exch{0.f, tot, 0.f, 0});
-    Z = 0.f;
-    for (int r = 0; r < c.C; ++r) {
-      rowtot[r] = got[r];
-      Z += got[r].f1;
-    }
-    if (gbad || !(Z > 0.f) || Z == INFINITY || M == -INFINITY) {
+    for (int r = 0; r < c.C; ++r) gtx = fmaxf(gtx, got[r].f2);
+    const float2 MZ = combine_ranks(got, c.C);
+    M = MZ.x;
+    Z = MZ.y;
+    // rank totals rescaled to the row maximum, for a placement on this row
+    // (a separate array: every thread is still reading `got` above)
+    if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
+    __syncthreads();
+    if (!(Z > 0.f) || Z == INFINITY || M == -INFINITY || M == INFINITY) {
       badrow = true;
       rejected = (j < L);
       y = 0;
@@ -431,10 +483,10 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     }
     if (j == L) {  // every verified draft accepted: bonus token from p of row L
       const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kBonus);
-      y = c.place(u * Z, [&](int i) { return exp2f(E::to_float(tb[i]) * cs - M); });
+      y = c.place(u * Z, M, [&](int i) { return ex2(fmaf(E::to_float(tb[i]), cs, -M)); });
       break;
     }
-    const float p = exp2f(gtx - M) / Z;
+    const float p = ex2(gtx - M) / Z;
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(j + 1), kAccept);
     if (!(u < p / a.q_tok[(long long)b * K + j])) {
       rejected = true;
@@ -446,42 +498,35 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   if (rejected && !greedy && !badrow) {
     // residual norm(max(0, p - q)) over target row acc (still in shared memory)
     // and draft row acc (q = softmax(d / temp), normaliser recomputed here)
-    bulk_load(db, drow0 + (long long)acc * V + c.lo, nbytes, &bar, phase, st, b);
-    float mq = -INFINITY;
-    c.each(db, [&](int, float v) { mq = fmaxf(mq, v); });
-    mq = c.block_max(mq) * cs;
-    c.gather(Exch{mq, 0.f, 0.f, 0});
-    float Mq = -INFINITY;
-    for (int r = 0; r < c.C; ++r) Mq = fmaxf(Mq, got[r].f0);
-    float sq = 0.f;
-    c.each(db, [&](int, float v) { sq += exp2f(v * cs - Mq); });
-    const float totq = c.block_scan_store(sq);
-    c.gather(Exch{0.f, totq, 0.f, 0});
-    float Zq = 0.f;
-    for (int r = 0; r < c.C; ++r) Zq += got[r].f1;
+    bulk_load(db, drow0 + (long long)acc * V + c.lo, nbytes, &bar, phase, st, b, &dead);
+    const float2 mq = c.online_stats(db, cs);
+    c.gather(Exch{mq.x, mq.y, 0.f, 0});
+    const float2 MZq = combine_ranks(got, c.C);
+    const float Mq = MZq.x, iZ = 1.f / Z, iZq = 1.f / MZq.y;
     auto resid_v = [&](float tv, float dv) {
-      const float p = exp2f(tv * cs - M) / Z;
-      const float q = exp2f(dv * cs - Mq) / Zq;
-      return fmaxf(0.f, p - q);
+      const float pp = ex2(fmaf(tv, cs, -M)) * iZ;
+      const float qq = ex2(fmaf(dv, cs, -Mq)) * iZq;
+      return fmaxf(0.f, pp - qq);
     };
     auto resid = [&](int i) { return resid_v(E::to_float(tb[i]), E::to_float(db[i])); };
     float sr = 0.f;
     c.each2(tb, db, [&](int, float tv, float dv) { sr += resid_v(tv, dv); });
-    const float totr = c.block_scan_store(sr);
+    const float totr = c.block_sum_keep(sr);
     c.gather(Exch{0.f, totr, 0.f, 0});
     float R = 0.f;
     for (int r = 0; r < c.C; ++r) R += got[r].f1;
+    if (tid < c.C) rw[tid] = got[tid].f1;
+    __syncthreads();
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kResidual);
     if (R > 0.f) {
-      y = c.place(u * R, resid);
+      y = c.place(u * R, 0.f, resid);
     } else {
       // exact-zero residual (floating point only): draw from p instead
-      float s = 0.f;
-      c.each(tb, [&](int, float v) { s += exp2f(v * cs - M); });
-      c.block_scan_store(s);
-      if (tid < c.C) got[tid] = rowtot[tid];
+      const float2 mz = c.online_stats(tb, cs);
+      c.gather(Exch{mz.x, mz.y, 0.f, 0});
+      if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
       __syncthreads();
-      y = c.place(u * Z, [&](int i) { return exp2f(E::to_float(tb[i]) * cs - M); });
+      y = c.place(u * Z, M, [&](int i) { return ex2(fmaf(E::to_float(tb[i]), cs, -M)); });
     }
   }
 

@@ -137,3 +137,23 @@ def test_round_replay_is_deterministic(cuda_ok):
     x1 = rnd.x.clone()
     rnd.run(dev, SEED, 10)  # a new round id draws new uniforms
     assert not torch.equal(rnd.x, x1)
+
+
+def test_masked_vocabulary_is_not_an_error(cuda_ok):
+    """Logits at -inf (masked tokens, here a quarter of the vocabulary spanning
+    whole chunks and CTA slices) weigh nothing: no status bit, never drawn, and
+    parity with the oracle holds."""
+    w = _small(B=24, V=8192)
+    inp = wl.generate(w)
+    masked = torch.zeros(w.V, dtype=torch.bool)
+    masked[1024:3072] = True
+    masked[::7] = True
+    inp["target"][:, :, masked] = float("-inf")
+    inp["base"][:, :, masked] = float("-inf")
+    for mode in (bn.CUT_COST, bn.CUT_NONE):
+        rnd, _ = run_gpu(w, inp, 3, mode)
+        check_round(w, inp, rnd, list(range(w.B)), 3, mode)
+        out = rnd.out.cpu()
+        emitted = out[out >= 0].long()
+        assert not masked[emitted].any()
+        assert not masked[rnd.x.cpu().long()].any()
