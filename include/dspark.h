@@ -182,6 +182,37 @@ int dspark_verify(const void* target, const void* d, const int32_t* x,
                   dspark_stream_t stream);
 
 /*
+ * dspark_draft_sample for callers that cannot allocate device memory. The pages
+ * have no counterpart to this entry point: it only changes where the scratch
+ * lives. dspark_draft_sample needs a caller-owned workspace; callers that run
+ * inside another runtime's memory manager (an inference server or framework
+ * whose caching allocator has reserved the device memory, so that an extra
+ * cudaMalloc can fail or upset its accounting), plug-in hosts that hand over
+ * only input and output buffers, and latency-critical paths that cannot accept
+ * cudaMalloc's implicit synchronisation have no way to provide one.
+ *
+ * Same arguments, computation and results as dspark_draft_sample, without
+ * ws/ws_bytes. The scratch is a fixed 8 MiB array inside the library's device
+ * image, held on every GPU that loads the library until the process exits; the
+ * call allocates and frees nothing. Its device address is looked up once per
+ * device, by the first call made while that device is current, so that first
+ * call should come before any stream capture. Every call uses the same array
+ * and clears its status part first: calls that overlap on the GPU (other
+ * streams, other threads) race and must not be issued. A call needs
+ * 256 + 8 * B * ceil(V / 256) bytes of the 8 MiB (B = 1024 at V = 151936 takes
+ * 4.9 MB); larger sizes return DSPARK_ERR_WORKSPACE.
+ *
+ *   status_out  [2] i32 device, out, or NULL: {OR of DSPARK_STATUS_* bits,
+ *               lowest offending request or -1} of this call
+ */
+int dspark_draft_sample_static(const void* base, const void* U, const void* W,
+                               const float* bias_scale, const int32_t* last_tok,
+                               const float* temp, int B, int K, int V, int r,
+                               int dtype, uint64_t seed, uint64_t round_id,
+                               int32_t* x, void* d, float* q_lse, float* q_tok,
+                               int32_t* status_out, dspark_stream_t stream);
+
+/*
  * Synchronises `stream`, reads the status block of `ws` into *code (OR of
  * DSPARK_STATUS_* bits) and *first_bad_request (-1 if none), then clears it.
  * Either output pointer may be NULL.

@@ -38,6 +38,8 @@ SIGNATURES = {
     "dspark_prefix_schedule": (_i, [_p, _p, _p, _f, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
                            _p, _sz, _p]),
+    "dspark_draft_sample_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
+                                        _p, _p, _p, _p, _p, _p]),
     "dspark_read_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32),
                                 ctypes.POINTER(ctypes.c_int32)]),
     "dspark_clear_status": (_i, [_p, _p]),
@@ -120,6 +122,23 @@ def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: in
         _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream))
     _check(rc, "dspark_draft_sample")
+
+
+def draft_sample_static(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: int,
+                        x, d, q_lse, q_tok, status_out=None, stream=None) -> None:
+    """dspark_draft_sample_static: dspark_draft_sample with the library's fixed
+    scratch instead of a workspace (for callers that cannot allocate)."""
+    B, K, V = base.shape
+    r = U.shape[1]
+    dt = _dtype_code(base)
+    rc = lib().dspark_draft_sample_static(
+        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
+        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
+        _ptr(temp, "temp", torch.float32), B, K, V, r, dt, seed, round_id,
+        _ptr(x, "x", torch.int32), _ptr(d, "d", base.dtype), _ptr(q_lse, "q_lse", torch.float32),
+        _ptr(q_tok, "q_tok", torch.float32), _ptr(status_out, "status_out", torch.int32),
+        _stream(stream))
+    _check(rc, "dspark_draft_sample_static")
 
 
 def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: int,
