@@ -14,9 +14,10 @@
 // 128-byte swizzle), D = fp32 in tensor memory (two 256-column buffers).
 //
 // Persistent CTAs, one per SM, warp-specialised:
-//   warp 0     TMA producer of W tiles (4-stage-per-tile ring of 32 KB stages)
+//   warp 0     TMA producer of W tiles (ring of four 16 KB stages of 32 ranks)
 //   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer
-//   warp 2     TMA producer of base tiles (ring of 16 KB [128 x 64] blocks)
+//   warp 2     TMA producer of base tiles (ring of six 16 KB [128 x 64] blocks,
+//              so the next tile's blocks load while this one is processed)
 //   warps 4-11 epilogue, two halves of four warps (one per TMEM lane
 //              quadrant): half h takes column blocks h and h+2 of every tile.
 //              tcgen05.ld of the accumulator (lane = request row), + base,
@@ -37,9 +38,11 @@ namespace tc {
 constexpr int kThreads = 384;      // 4 role warps + 8 epilogue warps
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
-constexpr int kWStages = 3;         // W ring depth (stages of 64 k-rows x 256 vocab)
-constexpr int kWStageBytes = 64 * 256 * 2;
-constexpr int kBaseSlots = 4;       // base/d blocks of one tile ([128 x 64] each)
+constexpr int kWRows = 32;          // Markov ranks per W stage
+constexpr int kWStages = 4;         // W ring depth (stages of 32 ranks x 256 vocab)
+constexpr int kWStageBytes = kWRows * 256 * 2;
+constexpr int kWBoxBytes = kWRows * 64 * 2;  // one [32 x 64] TMA box
+constexpr int kBaseSlots = 6;       // base/d ring of [128 x 64] blocks: 1.5 tiles
 constexpr int kBlockBytes = 128 * 64 * 2;
 constexpr int kABytes = 128 * 256 * 2;  // gathered U rows, 4 k-blocks of [128 x 64]
 
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt0 = blockIdx.x / p.m_per_launch;
   const int nstride = p.ctas_per_m;
   const int n_my = (nt0 < p.n_tiles) ? (p.n_tiles - nt0 + nstride - 1) / nstride : 0;
-  const int kblocks = (p.r + 63) / 64;   // W stages per tile
+  const int kblocks = (p.r + kWRows - 1) / kWRows;  // W stages per tile
   const int ksteps = p.r / 16;           // MMAs per tile
 
   if (tid == 0) {
@@ -269,7 +272,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&w_full[s], kWStageBytes);
         unsigned char* dst = sW + s * kWStageBytes;
 #pragma unroll
-        for (int vb = 0; vb < 4; ++vb) tma_load_2d(dst + vb * 8192, &map_w, n0 + vb * 64, kb * 64, &w_full[s]);
+        for (int vb = 0; vb < 4; ++vb)
+          tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + vb * 64, kb * kWRows, &w_full[s]);
         last[s] = it;
       }
       if (stop) break;
@@ -279,26 +283,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[q] >= 0) mbar_wait(&w_full[q], (last[q] / kWStages) & 1);
   } else if (warp == 2 && lane == 0) {
     // ---------------- base producer ----------------
-    // block j of every tile goes to ring slot j; the phase is the tile parity
-    int last_tile = -1;
-    for (int i = 0; i < n_my; ++i) {
-      const int n0 = (nt0 + i * nstride) * kTileN;
-      bool stop = false;
-      for (int j = 0; j < 4; ++j) {
-        if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[j], (i & 1) ^ 1)) {
-          if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcBaseEmpty, m0);
-          *(volatile int*)abort_flag = 1;
-          stop = true;
-          break;
-        }
-        mbar_expect_tx(&b_full[j], kBlockBytes);
-        tma_load_3d(sBase + j * kBlockBytes, &map_base, n0 + j * 64, p.k - 1, m0, &b_full[j]);
+    // block j of tile i is block g = 4i + j of the ring (slot g % kBaseSlots)
+    int last[kBaseSlots];
+    for (int q = 0; q < kBaseSlots; ++q) last[q] = -1;
+    for (int g = 0; g < 4 * n_my; ++g) {
+      const int s = g % kBaseSlots;
+      if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[s], ((g / kBaseSlots) & 1) ^ 1)) {
+        if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcBaseEmpty, m0);
+        *(volatile int*)abort_flag = 1;
+        break;
       }
-      last_tile = i;
-      if (stop) break;
+      const int n0 = (nt0 + (g >> 2) * nstride) * kTileN;
+      mbar_expect_tx(&b_full[s], kBlockBytes);
+      tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, p.k - 1, m0, &b_full[s]);
+      last[s] = g;
     }
-    if (*(volatile int*)abort_flag && last_tile >= 0)
-      for (int j = 0; j < 4; ++j) mbar_wait(&b_full[j], last_tile & 1);
+    if (*(volatile int*)abort_flag)
+      for (int q = 0; q < kBaseSlots; ++q)
+        if (last[q] >= 0) mbar_wait(&b_full[q], (last[q] / kBaseSlots) & 1);
   } else if (warp == 1 && lane == 0) {
     // ---------------- MMA issuer ----------------
     int it = 0;
@@ -324,13 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t w_base = su32(sW + s * kWStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const int step = kb * 4 + kk;
+        for (int kk = 0; kk < kWRows / 16; ++kk) {
+          const int step = kb * (kWRows / 16) + kk;  // 16 ranks per MMA
           if (step < ksteps) {
-            // A: k-block kb, 32-byte step kk inside the 128-byte swizzle row
-            const uint64_t ad = sdesc(a_base + kb * 16384 + kk * 32, 16, 1024);
-            // B: 16 k-rows (2 groups of 8) per step; 64-vocab blocks 8 KB apart
-            const uint64_t bd = sdesc(w_base + kk * 2048, 8192, 1024);
+            // A: 64-rank sub-tile step / 4, 32-byte step inside its 128-byte swizzle row
+            const uint64_t ad = sdesc(a_base + (step >> 2) * 16384 + (step & 3) * 32, 16, 1024);
+            // B: 16 k-rows (2 groups of 8) per step; 64-vocab boxes kWBoxBytes apart
+            const uint64_t bd = sdesc(w_base + kk * 2048, kWBoxBytes, 1024);
             const uint32_t acc = (step > 0) ? 1u : 0u;
             asm volatile(
                 "{\n .reg .pred pa;\n setp.ne.b32 pa, %4, 0;\n"
@@ -387,8 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       int arg = 0x7fffffff;
 #pragma unroll 1
       for (int jj = 0; jj < 2; ++jj) {
-        const int j = h + 2 * jj;       // column block, also its ring slot
-        if (!mbar_wait(&b_full[j], i & 1)) {
+        const int j = h + 2 * jj;       // column block of the tile
+        const int g = 4 * i + j;        // block of the ring
+        const int slot = g % kBaseSlots;
+        if (!mbar_wait(&b_full[slot], (g / kBaseSlots) & 1)) {
           miss = true;
           report_wait(p.status, kWhereTcBaseFull, m0);
         }
@@ -398,8 +402,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(col, acc);
         tmem_ld32(col + 32, acc + 32);
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        unsigned char* blk = sBase + j * kBlockBytes + row * 128;
+        unsigned char* blk = sBase + slot * kBlockBytes + row * 128;
         uint32_t dp[32];                // the block's 64 stored logits, packed
+        // d = round(base + sc * acc); the running maximum is taken on the
+        // unrounded sums: rounding to nearest is monotonic, so the rounded
+        // maximum is the maximum of the stored values (NaN propagates)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           uint4* ptr = reinterpret_cast<uint4*>(blk + ((c ^ (row & 7)) << 4));
@@ -410,6 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float y0 = fmaf(sc, acc[c * 8 + 2 * e], __uint_as_float(w[e] << 16));
             const float y1 = fmaf(sc, acc[c * 8 + 2 * e + 1], __uint_as_float(w[e] & 0xffff0000u));
             dp[c * 4 + e] = pack_bf16x2(y0, y1);
+            mx[e] = max_nan(mx[e], max_nan(y0, y1));
           }
           *ptr = make_uint4(dp[c * 4], dp[c * 4 + 1], dp[c * 4 + 2], dp[c * 4 + 3]);
         }
@@ -428,11 +437,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           } else {
-            float bm = -INFINITY;
+            float bm;
+            if (vcols == 64) {
+              const float m4 = max_nan(max_nan(mx[0], mx[1]), max_nan(mx[2], mx[3]));
+              bm = __uint_as_float(pack_bf16x2(m4, 0.f) << 16);  // = max of the stored values
+            } else {  // ragged last block: only the columns inside the vocabulary
+              bm = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 64; ++e) {
-              const float dv = __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16));
-              if (vcols == 64 || e < vcols) bm = max_nan(bm, dv);
+              for (int e = 0; e < 64; ++e)
+                if (e < vcols)
+                  bm = max_nan(bm, __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16)));
             }
             if (bm != bm) {
               run_s = NAN;  // a NaN logit: the chunk partial reports it
@@ -440,12 +454,22 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float nm = fmaxf(run_m, bm * cs);
               if (nm != -INFINITY) {  // -inf entries weigh nothing; +inf makes the sum NaN
                 const float neg = -nm;
-                float acc_s = 0.f;
+                float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+                if (vcols == 64) {
 #pragma unroll
-                for (int e = 0; e < 64; ++e) {
-                  const float dv = __uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u) : (dp[e >> 1] << 16));
-                  if (vcols == 64 || e < vcols) acc_s += ex2(fmaf(dv, cs, neg));
+                  for (int q2 = 0; q2 < 32; ++q2) {
+                    sacc[q2 & 3] += ex2(fmaf(__uint_as_float(dp[q2] << 16), cs, neg)) +
+                                    ex2(fmaf(__uint_as_float(dp[q2] & 0xffff0000u), cs, neg));
+                  }
+                } else {
+#pragma unroll
+                  for (int e = 0; e < 64; ++e)
+                    if (e < vcols)
+                      sacc[e & 3] += ex2(fmaf(__uint_as_float((e & 1) ? (dp[e >> 1] & 0xffff0000u)
+                                                                      : (dp[e >> 1] << 16)),
+                                              cs, neg));
                 }
+                const float acc_s = (sacc[0] + sacc[1]) + (sacc[2] + sacc[3]);
                 run_s = (run_m == -INFINITY ? 0.f : run_s * ex2(run_m - nm)) + acc_s;
               }
               run_m = nm;
@@ -456,13 +480,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         half_bar(h);
         if (elected) {
-          tma_store_3d(&map_d, sBase + j * kBlockBytes, n0 + j * 64, p.k - 1, m0);
+          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, p.k - 1, m0);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          mbar_arrive(&b_empty[j]);
+          if (jj == 1) {
+            // the first block's store has read its slot: hand it back; the
+            // second block's slot is handed back at the end of the tile
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            mbar_arrive(&b_empty[(4 * i + h) % kBaseSlots]);
+          }
         }
         __syncwarp();  // lane 0 may still be in the store above
       }
+      if (elected) {
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        mbar_arrive(&b_empty[(4 * i + h + 2) % kBaseSlots]);
+      }
+      __syncwarp();
       // this thread is done reading accumulator buffer `buf`
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&t_empty[buf]);
@@ -552,7 +585,7 @@ cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaS
   {
     const cuuint64_t dims[2] = {(cuuint64_t)a.V, (cuuint64_t)a.r};
     const cuuint64_t strides[1] = {(cuuint64_t)a.V * 2};
-    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kWRows};
     if (!make_map(&mw, a.W, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
