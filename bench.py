@@ -20,7 +20,6 @@ import os
 import subprocess
 import sys
 import time
-from datetime import timedelta
 
 import numpy as np
 import torch
@@ -29,6 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from speculative_decoding_draft_sample_b200 import binding as bn  # noqa: E402
+from speculative_decoding_draft_sample_b200 import replicas  # noqa: E402
 from speculative_decoding_draft_sample_b200 import workloads as wl  # noqa: E402
 from speculative_decoding_draft_sample_b200.spec_round import (DEVICE_KEYS, SpecRound,  # noqa: E402
                                                                 run_host, to_device)
@@ -100,40 +100,6 @@ class Clocks:
             return None
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm)}
-
-
-def dist_setup(n_gpus: int):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
-    else:
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-
-
-def max_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
-
-
-def sum_over_ranks(v: float, world: int) -> float:
-    if world == 1:
-        return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
 
 
 def time_region(fn, stream, iters: int) -> float:
@@ -217,12 +183,11 @@ def main():
         reference_arm(args, w)
         return
     assert args.warmup >= 3, "at least 3 warm-up steps"
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = replicas.init("nccl")
     hbm, tflops, tflops_sus, peak_kind = peaks()
 
     # each rank: its own batch (weak scaling), no collective on the data path
-    wr = wl.scaled(w, seed=rank) if rank else w
-    inp = wl.generate(wr)
+    inp = wl.generate(replicas.rank_workload(w, rank))
     dev = to_device(inp)
     rnd = SpecRound(w.B, w.K, w.V, w.r, torch.bfloat16)
     stream = torch.cuda.Stream()
@@ -255,7 +220,7 @@ def main():
     clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
     if clocks:
         clocks.start()
-    barrier(world)
+    replicas.barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -266,16 +231,16 @@ def main():
         e1.record(stream)
     e1.synchronize()
     torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    replicas.barrier()
+    ms = replicas.max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
     clk = clocks.stop() if clocks else None
 
     accepted = int(rnd.accepted.sum().item())
     emitted = int(rnd.n_emit.sum().item())
     cut = rnd.cut.cpu().numpy()
     acc_np = rnd.accepted.cpu().numpy()
-    acc_all = sum_over_ranks(float(accepted), world)
-    emit_all = sum_over_ranks(float(emitted), world)
+    acc_all = replicas.sum_over_ranks(float(accepted), "cuda")
+    emit_all = replicas.sum_over_ranks(float(emitted), "cuda")
     rounds_per_s = world * 1000.0 / ms
 
     # per-stage times (same stream, CUDA events), each stage alone
@@ -310,11 +275,11 @@ def main():
     with torch.cuda.stream(stream):
         for _ in range(2):
             run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, stream=stream)
-        barrier(world)
+        replicas.barrier()
         e2e_steps = max(3, args.steps // 5)
         ms_e2e = time_region(lambda: run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h,
                                               stream=stream), stream, e2e_steps)
-    ms_e2e = max_over_ranks(ms_e2e, world)
+    ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
     dominant = "verify" if ms_verify >= ms_draft / w.K else "draft"
     roof = {"kernel": "verify_kernel (dspark_verify)", "bound": "hbm", "achieved": verify_gbs,
@@ -348,10 +313,8 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), 128, 0).items()
                                 if k in ("value", "unit", "cores", "kind", "sample")}
-    del graph
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    del graph  # released before the process group goes away
+    replicas.finish()
     if rank == 0:
         print(json.dumps(line), flush=True)
 
