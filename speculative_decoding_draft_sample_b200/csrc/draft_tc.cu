@@ -90,28 +90,42 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t par) {
   return mbar_wait_bounded(su32(b), par);
 }
 
+// L2 eviction policies: W is re-read by every draft position (keep it), base
+// and d stream through once per position (let them go first).
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
-          su32(dst)),
-      "l"(map), "r"(su32(bar)), "r"(x), "r"(y)
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4}], [%2], %5;" ::"r"(su32(dst)),
+      "l"(map), "r"(su32(bar)), "r"(x), "r"(y), "l"(pol)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                            uint64_t* bar) {
+                                            uint64_t* bar, uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
-          su32(dst)),
-      "l"(map), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(su32(dst)),
+      "l"(map), "r"(su32(bar)), "r"(x), "r"(y), "r"(z), "l"(pol)
       : "memory");
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
-                                             int z) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   map),
-               "r"(su32(src)), "r"(x), "r"(y), "r"(z)
-               : "memory");
+                                             int z, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
+          map),
+      "r"(su32(src)), "r"(x), "r"(y), "r"(z), "l"(pol)
+      : "memory");
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -255,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     // ---------------- W producer ----------------
+    const uint64_t pol_w = policy_evict_last();
     int it = 0;
     int last[kWStages];
     for (int q = 0; q < kWStages; ++q) last[q] = -1;
@@ -273,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         unsigned char* dst = sW + s * kWStageBytes;
 #pragma unroll
         for (int vb = 0; vb < 4; ++vb)
-          tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + vb * 64, kb * kWRows, &w_full[s]);
+          tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + vb * 64, kb * kWRows, &w_full[s], pol_w);
         last[s] = it;
       }
       if (stop) break;
@@ -284,6 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2 && lane == 0) {
     // ---------------- base producer ----------------
     // block j of tile i is block g = 4i + j of the ring (slot g % kBaseSlots)
+    const uint64_t pol_base = policy_evict_first();
     int last[kBaseSlots];
     for (int q = 0; q < kBaseSlots; ++q) last[q] = -1;
     for (int g = 0; g < 4 * n_my; ++g) {
@@ -295,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int n0 = (nt0 + (g >> 2) * nstride) * kTileN;
       mbar_expect_tx(&b_full[s], kBlockBytes);
-      tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, p.k - 1, m0, &b_full[s]);
+      tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, p.k - 1, m0, &b_full[s], pol_base);
       last[s] = g;
     }
     if (*(volatile int*)abort_flag)
@@ -372,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc = (valid && p.bias_scale) ? p.bias_scale[b] : 1.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool elected = (warp == 4 + 4 * h) && lane == 0;
+    const uint64_t pol_d = policy_evict_first();
     bool miss = false;
     for (int i = 0; i < n_my; ++i) {
       const int nt = nt0 + i * nstride;
@@ -480,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         half_bar(h);
         if (elected) {
-          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, p.k - 1, m0);
+          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, p.k - 1, m0, pol_d);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           if (jj == 1) {
             // the first block's store has read its slot: hand it back; the

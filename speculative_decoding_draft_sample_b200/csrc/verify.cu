@@ -9,21 +9,26 @@
 // inference speedup", "Speculative Decoding in Two Sentences": one bonus token
 // is appended when the whole verified block is accepted.
 //
-// Design (B200): one thread-block cluster of C CTAs per request; CTA `rank`
-// owns vocabulary slice [rank*slice, rank*slice + slice). The request's target
-// rows are walked in order and the walk stops at the first rejection, so only
-// rows 0..a and one draft row are ever read. Each row slice lands in shared
-// memory with one bulk asynchronous copy (cp.async.bulk, completion on an
-// mbarrier); every reduction across the cluster goes through distributed
-// shared memory. The residual pass re-reads the target row from shared memory,
-// so HBM sees every byte once.
+// Design (B200): one thread-block cluster of C small CTAs (128 threads) per
+// request; CTA `rank` owns vocabulary slice [rank*slice, rank*slice + slice).
+// A request's target rows are walked in order and the walk stops at the first
+// rejection, so HBM sees only rows 0..a and one draft row. Each slice streams
+// through a ring of 4 KB shared-memory slots filled by bulk asynchronous copies
+// (cp.async.bulk, completion on mbarriers): no row is kept resident, so a CTA
+// needs 17 KB of shared memory and every request of the batch is in flight at
+// once. One online (max, sum 2^z) pass per row and one exchange over
+// distributed shared memory give the row's normaliser; only the CTA that owns
+// an inverse-CDF crossing streams its slice again (from L2) to place the token.
 #include "common.cuh"
 #include "verify.cuh"
 
 namespace dspark {
 
-constexpr int kVThreads = 256;
-constexpr int kMaxCluster = 8;
+constexpr int kVThreads = 128;
+constexpr int kVBlocksPerSM = 8;
+constexpr int kSlotBytes = 4096;
+constexpr int kRing = 4;
+constexpr int kMaxCluster = 16;
 
 // One value each CTA publishes to its cluster per exchange.
 struct __align__(16) Exch {
@@ -64,44 +69,13 @@ __device__ __forceinline__ uint4 dsmem_load16(const void* local, int rank) {
   return v;
 }
 
-// Bulk copy of `bytes` (multiple of 16) from global to this CTA's shared memory,
-// completing on `bar`; every thread then waits (bounded) for phase `phase`.
-__device__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
-                          uint32_t& phase, Status* st, int request, int* dead) {
-  if (*(volatile int*)dead) {  // this CTA already gave up once: no more copies or waits
-    phase ^= 1u;
-    return;
-  }
-  const uint32_t b = smem_u32(bar);
-  if (threadIdx.x == 0) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
-                 : "memory");
-    for (uint32_t off = 0; off < bytes; off += 16384) {
-      const uint32_t n = min(16384u, bytes - off);
-      asm volatile(
-          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-              smem_u32(static_cast<char*>(dst) + off)),
-          "l"(static_cast<const char*>(src) + off), "r"(n), "r"(b)
-          : "memory");
-    }
-  }
-  if (!mbar_wait_bounded(b, phase)) {
-    if (threadIdx.x == 0) report_wait(st, kWhereVerifyLoad, request);
-    mbar_wait_bounded(b, phase);  // give an in-flight copy a last chance to land
-    *(volatile int*)dead = 1;
-  }
-  __syncwarp();
-  __syncthreads();  // every thread sees the same `dead` before the next copy
-  phase ^= 1u;
-}
-
 // 16 bytes of shared memory as floats (8 bf16 or 4 fp32), in index order.
 template <int DT>
 struct Vec16;
 template <>
 struct Vec16<DSPARK_BF16> {
   static constexpr int N = 8;
-  __device__ __forceinline__ static void load(const uint16_t* p, float* v) {
+  __device__ __forceinline__ static void load(const void* p, float* v) {
     const uint4 q = *reinterpret_cast<const uint4*>(p);
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
@@ -114,7 +88,7 @@ struct Vec16<DSPARK_BF16> {
 template <>
 struct Vec16<DSPARK_F32> {
   static constexpr int N = 4;
-  __device__ __forceinline__ static void load(const float* p, float* v) {
+  __device__ __forceinline__ static void load(const void* p, float* v) {
     const float4 q = *reinterpret_cast<const float4*>(p);
     v[0] = q.x;
     v[1] = q.y;
@@ -123,22 +97,109 @@ struct Vec16<DSPARK_F32> {
   }
 };
 
+// Combines the online pair (m2, s2) into (m, s); NaN propagates.
+__device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
+  const float mm = fmaxf(m, m2);
+  const float a = (m == -INFINITY) ? 0.f : s * ex2(m - mm);
+  const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2(m2 - mm);
+  s = (s != s || s2 != s2) ? NAN : a + b;
+  m = mm;
+}
+
 template <int DT>
 struct VerifyCta {
   using E = Elem<DT>;
   using T = typename E::T;
+  static constexpr int N = Vec16<DT>::N;            // elements per 16-byte vector
+  static constexpr int kStepElems = kSlotBytes / E::kBytes;
 
   int C, rank, tid, lane, warp;
-  int lo, n, per, t0, t1;  // slice [lo, lo+n); this thread's elements [t0, t1) of it
+  int lo, n;               // slice [lo, lo + n) of the vocabulary
+  unsigned char* ring;     // kRing slots of kSlotBytes
+  uint64_t* bars;          // kRing mbarriers
   Exch* ex;                // [2] published slots (double buffered)
   Exch* got;               // [kMaxCluster] gathered copies (read-only after a gather)
-  float* rw;               // [kMaxCluster] per-rank weights of the placement at hand
-  float* pm;               // [kVThreads] per-thread running max (online rows)
-  float* ps;               // [kVThreads] per-thread sums
-  float* excl;             // [kVThreads] exclusive block scan of the weights
   float* red;              // [32] scratch
   int* sint;               // [4] scratch
+  int* dead;               // set once a wait gave up
+  Status* st;
+  int request;
   int parity;
+  uint32_t issued, consumed;  // ring slot counters (identical in every thread)
+
+  // ---------------- streaming through the ring ----------------
+  __device__ void issue(const T* src, uint32_t bytes) {
+    const uint32_t r = issued % kRing;
+    if (threadIdx.x == 0 && !*(volatile int*)dead) {
+      const uint32_t b = smem_u32(&bars[r]);
+      // generic reads of the slot's previous contents are barrier-ordered before this
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+              smem_u32(ring + r * kSlotBytes)),
+          "l"(src), "r"(bytes), "r"(b)
+          : "memory");
+    }
+    ++issued;
+  }
+  __device__ const unsigned char* wait() {
+    const uint32_t r = consumed % kRing;
+    const uint32_t ph = (consumed / kRing) & 1u;
+    if (!*(volatile int*)dead && !mbar_wait_bounded(smem_u32(&bars[r]), ph)) {
+      if (threadIdx.x == 0) report_wait(st, kWhereVerifyLoad, request);
+      mbar_wait_bounded(smem_u32(&bars[r]), ph);  // a last chance for an in-flight copy
+      *(volatile int*)dead = 1;
+    }
+    __syncwarp();
+    ++consumed;
+    return ring + r * kSlotBytes;
+  }
+  __device__ int steps() const { return (n + kStepElems - 1) / kStepElems; }
+  __device__ uint32_t step_bytes(int s) const {
+    return (uint32_t)min(kStepElems, n - s * kStepElems) * E::kBytes;
+  }
+
+  // One pass over `nrow` (1 or 2) row slices, step by step; f(step, slot0,
+  // slot1) runs in every thread once a step's slots have landed and must be
+  // done with them when it returns. f returns true to stop the pass early (the
+  // copies still in flight are drained).
+  template <class F>
+  __device__ void pass(const T* r0, const T* r1, int nrow, F f) {
+    const int ns = steps();
+    const int ahead = kRing / nrow;
+    int next = 0;
+    for (; next < ns && next < ahead; ++next) {
+      issue(r0 + next * kStepElems, step_bytes(next));
+      if (nrow == 2) issue(r1 + next * kStepElems, step_bytes(next));
+    }
+    int s = 0;
+    while (s < ns) {
+      const unsigned char* a = wait();
+      const unsigned char* b = (nrow == 2) ? wait() : nullptr;
+      __syncthreads();  // every thread sees the landed bytes and `dead`
+      const bool stop = f(s, a, b);
+      __syncthreads();  // the slots are free again
+      ++s;
+      if (stop) break;
+      if (next < ns) {
+        issue(r0 + next * kStepElems, step_bytes(next));
+        if (nrow == 2) issue(r1 + next * kStepElems, step_bytes(next));
+        ++next;
+      }
+    }
+    for (int k = s; k < next; ++k) {  // drain an early stop
+      wait();
+      if (nrow == 2) wait();
+    }
+    __syncthreads();
+  }
+
+  // first element of this thread's vector h (0 or 1) of step s
+  __device__ __forceinline__ int vec_elem(int s, int h) const {
+    return s * kStepElems + (tid + h * kVThreads) * N;
+  }
 
   // Publishes this CTA's value and gathers every CTA's (one cluster barrier).
   __device__ void gather(const Exch& mine) {
@@ -152,106 +213,92 @@ struct VerifyCta {
     parity ^= 1;
   }
 
-  // f(i, value) over this thread's elements of `buf`, in index order, 16 B at a time
-  template <class F>
-  __device__ __forceinline__ void each(const T* buf, F f) const {
-    constexpr int N = Vec16<DT>::N;
-    for (int i = t0; i < t1; i += N) {
-      float v[N];
-      Vec16<DT>::load(buf + i, v);
+  // CTA-wide online (max, sum) of the per-thread pairs
+  __device__ float2 block_online(float m, float s) {
 #pragma unroll
-      for (int j = 0; j < N; ++j) f(i + j, v[j]);
-    }
-  }
-  template <class F>
-  __device__ __forceinline__ void each2(const T* b1, const T* b2, F f) const {
-    constexpr int N = Vec16<DT>::N;
-    for (int i = t0; i < t1; i += N) {
-      float v1[N], v2[N];
-      Vec16<DT>::load(b1 + i, v1);
-      Vec16<DT>::load(b2 + i, v2);
-#pragma unroll
-      for (int j = 0; j < N; ++j) f(i + j, v1[j], v2[j]);
-    }
-  }
-
-  // Online (max, sum 2^(z - max)) of z = v * cs over this thread's elements,
-  // kept in pm/ps for a later placement; returns the CTA's pair (thread 0's
-  // result is the one published). NaN or +inf anywhere makes the sum NaN.
-  __device__ float2 online_stats(const T* buf, float cs) {
-    constexpr int N = Vec16<DT>::N;
-    float m = -INFINITY, sum = 0.f;
-    for (int i = t0; i < t1; i += N) {
-      float v[N];
-      Vec16<DT>::load(buf + i, v);
-      float vm = v[0];
-#pragma unroll
-      for (int j = 1; j < N; ++j) vm = max_nan(vm, v[j]);
-      const float zm = vm * cs;
-      if (zm != zm) {  // NaN in this vector
-        sum = NAN;
-        continue;
-      }
-      if (zm > m) {
-        sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
-        m = zm;
-      }
-      if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
-        const float neg = -m;
-#pragma unroll
-        for (int j = 0; j < N; ++j) sum += ex2(fmaf(v[j], cs, neg));
-      }
-    }
-    pm[tid] = m;
-    ps[tid] = sum;
-    // warp combine, then the 8 warp results
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-      const float s2 = __shfl_xor_sync(0xffffffffu, sum, o);
-      const float mm = fmaxf(m, m2);
-      const float a = (m == -INFINITY) ? 0.f : sum * ex2(m - mm);
-      const float b = (m2 == -INFINITY) ? 0.f : s2 * ex2(m2 - mm);
-      sum = (sum != sum || s2 != s2) ? NAN : a + b;
-      m = mm;
-    }
+    for (int o = 16; o; o >>= 1)
+      online_merge(m, s, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, s, o));
     if (lane == 0) {
       red[warp] = m;
-      red[8 + warp] = sum;
+      red[8 + warp] = s;
     }
     __syncthreads();
     float M = red[0], S = red[8];
-    for (int w = 1; w < kVThreads / 32; ++w) {
-      const float mm = fmaxf(M, red[w]);
-      const float a = (M == -INFINITY) ? 0.f : S * ex2(M - mm);
-      const float b = (red[w] == -INFINITY) ? 0.f : red[8 + w] * ex2(red[w] - mm);
-      S = (S != S || red[8 + w] != red[8 + w]) ? NAN : a + b;
-      M = mm;
-    }
+    for (int w = 1; w < kVThreads / 32; ++w) online_merge(M, S, red[w], red[8 + w]);
     __syncthreads();
     return make_float2(M, S);
   }
-
-  // Block sum of per-thread values (also kept in ps for a later placement).
-  __device__ float block_sum_keep(float v) {
-    ps[tid] = v;
-    pm[tid] = 0.f;  // weights are ps * 2^(pm - 0)
-    const float w = warp_sum(v);
-    if (lane == 0) red[warp] = w;
+  __device__ float block_sum(float v) {
+    v = warp_sum(v);
+    if (lane == 0) red[warp] = v;
     __syncthreads();
     float t = 0.f;
-    for (int i = 0; i < kVThreads / 32; ++i) t += red[i];
+    for (int w = 0; w < kVThreads / 32; ++w) t += red[w];
     __syncthreads();
     return t;
   }
 
-  // Inverse-CDF placement of `thr` on weights wfun(i) (slice-local index i).
-  // Per-rank totals are rw[r]; this thread's total weight is
-  // ps[tid] * 2^(pm[tid] - Mref). Returns the global token index in every
-  // thread of the owning CTA, -1 in the other CTAs, and -2 everywhere if no
-  // rank holds positive mass. No cluster exchange happens here.
+  // CTA-wide online (max, sum 2^(z - max)) of z = v * cs over the slice of `row`.
+  __device__ float2 row_stats(const T* row, float cs) {
+    float m = -INFINITY, sum = 0.f;
+    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (vec_elem(s, h) >= n) continue;
+        float v[N];
+        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, v);
+        float vm = v[0];
+#pragma unroll
+        for (int j = 1; j < N; ++j) vm = max_nan(vm, v[j]);
+        const float zm = vm * cs;
+        if (zm != zm) {  // NaN in this vector
+          sum = NAN;
+          continue;
+        }
+        if (zm > m) {
+          sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
+          m = zm;
+        }
+        if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
+          const float neg = -m;
+#pragma unroll
+          for (int j = 0; j < N; ++j) sum += ex2(fmaf(v[j], cs, neg));
+        }
+      }
+      return false;
+    });
+    return block_online(m, sum);
+  }
+
+  // Per-thread (max, lowest argmax) of the raw values and a NaN / +inf check.
+  __device__ void row_argmax(const T* row, float& mv, int& mi, float& chk) {
+    mv = -INFINITY;
+    mi = 0x7fffffff;
+    chk = -INFINITY;
+    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int e0 = vec_elem(s, h);
+        if (e0 >= n) continue;
+        float v[N];
+        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, v);
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          chk = max_nan(chk, v[j]);
+          argmax_merge(mv, mi, v[j], lo + e0 + j);
+        }
+      }
+      return false;
+    });
+  }
+
+  // Inverse-CDF placement of `thr` on the weights wfun(t_value, d_value) of the
+  // cluster's slices, in index order. rw[r] are the per-rank totals (identical
+  // in every CTA). Only the owning CTA streams its slice again; it returns the
+  // token in every thread, the other CTAs return -1, and -2 means that no rank
+  // holds positive mass. No cluster exchange happens here.
   template <class F>
-  __device__ int place(float thr, float Mref, F wfun) {
+  __device__ int place(float thr, const float* rw, const T* r0, const T* r1, int nrow, F wfun) {
     int owner = -1, lastpos = -1;
     float P = 0.f, Pown = 0.f;
     for (int r = 0; r < C; ++r) {
@@ -272,50 +319,89 @@ struct VerifyCta {
     }
     if (owner < 0) return -2;
     if (owner != rank) return -1;
-    // this thread's weight and its exclusive prefix in index order
-    const float wt = (pm[tid] == -INFINITY) ? 0.f : ps[tid] * ex2(pm[tid] - Mref);
-    const float incl = warp_inclusive_scan(wt);
-    if (lane == 31) red[warp] = incl;
+    float rem = fallback ? INFINITY : thr - Pown;
+    int found = -1;
+    int lastp = -1;  // last element of positive weight this thread has seen
+    if (tid == 0) sint[0] = -1;
     __syncthreads();
-    float pre = 0.f;
-    for (int w = 0; w < warp; ++w) pre += red[w];
-    const float ex_t = pre + incl - wt;
-    const float rem = fallback ? INFINITY : thr - Pown;
-    if (tid == 0) sint[1] = 0x7fffffff;
-    __syncthreads();
-    if (wt > 0.f && rem < ex_t + wt) atomicMin(&sint[1], tid);
-    __syncthreads();
-    int ot = sint[1];
-    bool tfall = fallback;
-    if (ot == 0x7fffffff) {  // rounding: last thread with positive mass
+    pass(r0, r1, nrow, [&](int s, const unsigned char* a, const unsigned char* b) {
+      float vs[2], w[2][N];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        vs[h] = 0.f;
+#pragma unroll
+        for (int j = 0; j < N; ++j) w[h][j] = 0.f;
+        const int e0 = vec_elem(s, h);
+        if (e0 >= n) continue;
+        float tv[N], dv[N];
+        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, tv);
+        if (b) Vec16<DT>::load(b + (tid + h * kVThreads) * 16, dv);
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          w[h][j] = wfun(tv[j], b ? dv[j] : 0.f);
+          vs[h] += w[h][j];
+          if (w[h][j] > 0.f) lastp = e0 + j;
+        }
+      }
+      // exclusive prefix of the vectors' sums over the step (vector k = h * 128 + tid)
+      float pre[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float incl = warp_inclusive_scan(vs[h]);
+        if (lane == 31) red[h * 4 + warp] = incl;
+        pre[h] = incl - vs[h];
+      }
+      __syncthreads();
+      float base[2], tot = 0.f, half0 = 0.f;
+      base[0] = pre[0];
+      base[1] = pre[1];
+      for (int k = 0; k < 4; ++k) {
+        half0 += red[k];
+        if (k < warp) {
+          base[0] += red[k];
+          base[1] += red[4 + k];
+        }
+      }
+      base[1] += half0;
+      for (int k = 0; k < 8; ++k) tot += red[k];
+      if (!(rem < tot)) {
+        rem -= tot;
+        return false;
+      }
+      // the crossing is in this step: the first vector whose range holds it
+      if (tid == 0) sint[1] = 0x7fffffff;
+      __syncthreads();
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        if (vs[h] > 0.f && rem < base[h] + vs[h]) atomicMin(&sint[1], h * kVThreads + tid);
+      __syncthreads();
+      const int kv = sint[1];
+      if (kv != 0x7fffffff && (kv % kVThreads) == tid) {
+        const int h = kv / kVThreads;
+        float r2 = rem - base[h];
+        int f = -1, lp = -1;
+#pragma unroll
+        for (int j = 0; j < N; ++j) {
+          if (w[h][j] > 0.f) lp = j;
+          if (f < 0 && r2 < w[h][j]) f = j;
+          if (f < 0) r2 -= w[h][j];
+        }
+        if (f < 0) f = lp;
+        sint[0] = vec_elem(s, h) + max(f, 0);
+      }
+      __syncthreads();
+      found = sint[0];
+      if (found < 0) rem -= tot;  // rounding: no vector held it; the fallback below decides
+      return found >= 0;
+    });
+    if (found < 0) {  // no crossing (rounding only): the last element of positive weight
       if (tid == 0) sint[2] = -1;
       __syncthreads();
-      if (wt > 0.f) atomicMax(&sint[2], tid);
+      atomicMax(&sint[2], lastp);
       __syncthreads();
-      ot = sint[2];
-      tfall = true;
+      found = max(sint[2], 0);
     }
-    if (tid == 0) sint[3] = -1;
-    __syncthreads();
-    if (tid == ot) {
-      float r2 = tfall ? INFINITY : rem - ex_t;
-      int found = -1, lastp = -1;
-      for (int i = t0; i < t1; ++i) {
-        const float w = wfun(i);
-        if (w > 0.f) lastp = i;
-        if (r2 < w) {
-          found = i;
-          break;
-        }
-        r2 -= w;
-      }
-      if (found < 0) found = lastp;
-      sint[3] = found;
-    }
-    __syncthreads();
-    const int f = sint[3];
-    __syncthreads();
-    return f < 0 ? lo : lo + f;
+    return lo + found;
   }
 };
 
@@ -333,16 +419,16 @@ __device__ __forceinline__ float2 combine_ranks(const Exch* got, int C) {
 }
 
 template <int DT>
-__global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
+__global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(VerifyArgs a) {
   using E = Elem<DT>;
   using T = typename E::T;
-  extern __shared__ __align__(128) unsigned char dsm[];
+  __shared__ __align__(128) unsigned char ring[kRing * kSlotBytes];
+  __shared__ __align__(8) uint64_t bars[kRing];
   __shared__ Exch ex[2];
   __shared__ Exch got[kMaxCluster];
   __shared__ float rw[kMaxCluster];
-  __shared__ float pm[kVThreads], ps[kVThreads], excl[kVThreads], red[32];
+  __shared__ float red[32];
   __shared__ int sint[4];
-  __shared__ __align__(8) uint64_t bar;
   __shared__ int dead;
 
   VerifyCta<DT> c;
@@ -351,41 +437,31 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   c.tid = threadIdx.x;
   c.lane = c.tid & 31;
   c.warp = c.tid >> 5;
+  c.ring = ring;
+  c.bars = bars;
   c.ex = ex;
   c.got = got;
-  c.rw = rw;
-  c.pm = pm;
-  c.ps = ps;
-  c.excl = excl;
   c.red = red;
   c.sint = sint;
+  c.dead = &dead;
+  c.st = a.status;
   c.parity = 0;
+  c.issued = 0;
+  c.consumed = 0;
   const int b = blockIdx.x / c.C;
+  c.request = b;
   c.lo = c.rank * a.slice;
   c.n = max(0, min(a.slice, a.V - c.lo));
-  {
-    // each thread: a contiguous run of an odd number of 16-byte chunks, so that
-    // the 16-byte shared-memory loads of a quarter warp fall in distinct banks
-    constexpr int v16 = Vec16<DT>::N;
-    int per = (c.n + kVThreads - 1) / kVThreads;
-    per = (per + v16 - 1) / v16 * v16;
-    if (((per / v16) & 1) == 0) per += v16;
-    c.per = per;
-  }
-  c.t0 = min(c.tid * c.per, c.n);
-  c.t1 = min(c.t0 + c.per, c.n);
-  T* tb = reinterpret_cast<T*>(dsm);
-  T* db = reinterpret_cast<T*>(dsm + a.slice_bytes_padded);
   Status* st = a.status;
   const int tid = c.tid;
 
   if (tid == 0) {
     dead = 0;
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bar)) : "memory");
+    for (int i = 0; i < kRing; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])) : "memory");
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  uint32_t phase = 0;
 
   const int K = a.K, V = a.V;
   int L = a.cut ? a.cut[b] : K;
@@ -401,7 +477,6 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   const float cs = greedy ? 1.f : kLog2e / tau;
   const T* target = static_cast<const T*>(a.target) + (long long)b * (K + 1) * V;
   const T* drow0 = static_cast<const T*>(a.d) + (long long)b * K * V;
-  const uint32_t nbytes = (uint32_t)c.n * E::kBytes;
 
   int acc = 0;
   bool rejected = false;
@@ -410,19 +485,13 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   int y = -1;
 
   for (int j = 0; j <= L; ++j) {
-    bulk_load(tb, target + (long long)j * V + c.lo, nbytes, &bar, phase, st, b, &dead);
+    const T* row = target + (long long)j * V;
     const int xk = (j < L) ? a.x[(long long)b * K + j] : -1;
     if (j < L && (xk < 0 || xk >= V) && tid == 0 && c.rank == 0) report(st, DSPARK_STATUS_BAD_TOKEN, b);
     if (greedy) {
-      float mv = -INFINITY, chk = -INFINITY;
-      int mi = 0x7fffffff;
-      c.each(tb, [&](int i, float v) {
-        chk = max_nan(chk, v);
-        if (v > mv) {
-          mv = v;
-          mi = c.lo + i;
-        }
-      });
+      float mv, chk;
+      int mi;
+      c.row_argmax(row + c.lo, mv, mi, chk);
       warp_argmax(mv, mi);
 #pragma unroll
       for (int o = 16; o; o >>= 1) chk = max_nan(chk, __shfl_xor_sync(0xffffffffu, chk, o));
@@ -461,10 +530,11 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
       continue;
     }
 
-    // one online pass: (max, sum) of z = t * cs, and t[x] of the draft tested
-    const float2 mz = c.online_stats(tb, cs);
+    // one online pass: (max, sum) of z = t * cs; t[x] of the draft being tested
+    // comes from the CTA whose slice holds x
+    const float2 mz = c.row_stats(row + c.lo, cs);
     float tx = -INFINITY;
-    if (xk >= c.lo && xk < c.lo + c.n) tx = E::to_float(tb[xk - c.lo]) * cs;
+    if (tid == 0 && xk >= c.lo && xk < c.lo + c.n) tx = E::load(row, xk) * cs;
     c.gather(Exch{mz.x, mz.y, tx, 0});
     float gtx = -INFINITY;
     for (int r = 0; r < c.C; ++r) gtx = fmaxf(gtx, got[r].f2);
@@ -483,7 +553,8 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     }
     if (j == L) {  // every verified draft accepted: bonus token from p of row L
       const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kBonus);
-      y = c.place(u * Z, M, [&](int i) { return ex2(fmaf(E::to_float(tb[i]), cs, -M)); });
+      y = c.place(u * Z, rw, row + c.lo, nullptr, 1,
+                  [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); });
       break;
     }
     const float p = ex2(gtx - M) / Z;
@@ -496,22 +567,34 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
   }
 
   if (rejected && !greedy && !badrow) {
-    // residual norm(max(0, p - q)) over target row acc (still in shared memory)
-    // and draft row acc (q = softmax(d / temp), normaliser recomputed here)
-    bulk_load(db, drow0 + (long long)acc * V + c.lo, nbytes, &bar, phase, st, b, &dead);
-    const float2 mq = c.online_stats(db, cs);
+    // residual norm(max(0, p - q)) over target row acc and draft row acc
+    // (q = softmax(d / temp), its normaliser recomputed here)
+    const T* trow = target + (long long)acc * V + c.lo;
+    const T* drow = drow0 + (long long)acc * V + c.lo;
+    const float2 mq = c.row_stats(drow, cs);
     c.gather(Exch{mq.x, mq.y, 0.f, 0});
     const float2 MZq = combine_ranks(got, c.C);
     const float Mq = MZq.x, iZ = 1.f / Z, iZq = 1.f / MZq.y;
-    auto resid_v = [&](float tv, float dv) {
+    auto resid = [&](float tv, float dv) {
       const float pp = ex2(fmaf(tv, cs, -M)) * iZ;
       const float qq = ex2(fmaf(dv, cs, -Mq)) * iZq;
       return fmaxf(0.f, pp - qq);
     };
-    auto resid = [&](int i) { return resid_v(E::to_float(tb[i]), E::to_float(db[i])); };
     float sr = 0.f;
-    c.each2(tb, db, [&](int, float tv, float dv) { sr += resid_v(tv, dv); });
-    const float totr = c.block_sum_keep(sr);
+    c.pass(trow, drow, 2, [&](int s, const unsigned char* ta, const unsigned char* da) {
+      constexpr int N = Vec16<DT>::N;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (c.vec_elem(s, h) >= c.n) continue;
+        float tv[N], dv[N];
+        Vec16<DT>::load(ta + (tid + h * kVThreads) * 16, tv);
+        Vec16<DT>::load(da + (tid + h * kVThreads) * 16, dv);
+#pragma unroll
+        for (int j = 0; j < N; ++j) sr += resid(tv[j], dv[j]);
+      }
+      return false;
+    });
+    const float totr = c.block_sum(sr);
     c.gather(Exch{0.f, totr, 0.f, 0});
     float R = 0.f;
     for (int r = 0; r < c.C; ++r) R += got[r].f1;
@@ -519,14 +602,14 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
     __syncthreads();
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kResidual);
     if (R > 0.f) {
-      y = c.place(u * R, 0.f, resid);
+      y = c.place(u * R, rw, trow, drow, 2, resid);
     } else {
       // exact-zero residual (floating point only): draw from p instead
-      const float2 mz = c.online_stats(tb, cs);
+      const float2 mz = c.row_stats(trow, cs);
       c.gather(Exch{mz.x, mz.y, 0.f, 0});
       if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
       __syncthreads();
-      y = c.place(u * Z, M, [&](int i) { return ex2(fmaf(E::to_float(tb[i]), cs, -M)); });
+      y = c.place(u * Z, rw, trow, nullptr, 1, [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); });
     }
   }
 
@@ -551,22 +634,24 @@ __global__ void __launch_bounds__(kVThreads) verify_kernel(VerifyArgs a) {
 }
 
 int verify_cluster_size(int B, int V, int dtype, int num_sms) {
-  // Aim for a few CTAs per SM and row slices of at most ~40 KB, with at most
-  // kMaxCluster CTAs per request.
-  const long long row_bytes = (long long)V * (dtype == DSPARK_F32 ? 4 : 2);
+  // Enough CTAs in flight to keep HBM busy (kVBlocksPerSM 128-thread CTAs per
+  // SM), at most 16 per request, and at least one ring step per CTA.
+  const int es = dtype == DSPARK_F32 ? 4 : 2;
+  const long long slots = (long long)kVBlocksPerSM * num_sms;
   int C = 1;
-  while (C < kMaxCluster && (row_bytes / C > 40 * 1024 || (long long)B * C < 2LL * num_sms)) C <<= 1;
+  while (C < kMaxCluster && (long long)B * C * 2 <= slots &&
+         (long long)V * es / (2 * C) >= kSlotBytes)
+    C <<= 1;
   return C;
 }
 
 size_t verify_smem_bytes(int V, int dtype, int C, int* slice, size_t* slice_padded) {
-  const int es = dtype == DSPARK_F32 ? 4 : 2;
+  (void)dtype;
   int s = (V + C - 1) / C;
   s = (s + 7) & ~7;
-  const size_t sb = ((size_t)s * es + 127) & ~(size_t)127;
   if (slice) *slice = s;
-  if (slice_padded) *slice_padded = sb;
-  return 2 * sb;
+  if (slice_padded) *slice_padded = 0;
+  return 0;  // the 16 KB ring and the bookkeeping are static shared memory
 }
 
 cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s) {
@@ -574,8 +659,10 @@ cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s) {
   const size_t sm = verify_smem_bytes(a.V, a.dtype, C, &a.slice, &padded);
   a.slice_bytes_padded = padded;
   auto kern = (a.dtype == DSPARK_F32) ? verify_kernel<DSPARK_F32> : verify_kernel<DSPARK_BF16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
-  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.B * C));
   cfg.blockDim = dim3(kVThreads);
@@ -588,8 +675,7 @@ cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, a);
-  return e;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 }  // namespace dspark
