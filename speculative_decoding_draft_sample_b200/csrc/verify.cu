@@ -13,10 +13,11 @@
 // request; CTA `rank` owns vocabulary slice [rank*slice, rank*slice + slice).
 // A request's target rows are walked in order and the walk stops at the first
 // rejection, so HBM sees only rows 0..a and one draft row. Each slice streams
-// through a ring of 4 KB shared-memory slots filled by bulk asynchronous copies
-// (cp.async.bulk, completion on mbarriers): no row is kept resident, so a CTA
-// needs 17 KB of shared memory and every request of the batch is in flight at
-// once. One online (max, sum 2^z) pass per row and one exchange over
+// through a ring of 8 KB shared-memory slots filled by bulk asynchronous copies
+// (cp.async.bulk; a "full" mbarrier per slot completes with the bytes, a
+// per-warp "empty" arrival hands the slot back): no row is kept resident, so a
+// CTA needs 33 KB of shared memory and every request of the batch is in flight
+// at once. One online (max, sum 2^z) pass per row and one exchange over
 // distributed shared memory give the row's normaliser; only the CTA that owns
 // an inverse-CDF crossing streams its slice again (from L2) to place the token.
 #include "common.cuh"
@@ -25,9 +26,10 @@
 namespace dspark {
 
 constexpr int kVThreads = 128;
-constexpr int kVBlocksPerSM = 8;
-constexpr int kSlotBytes = 4096;
+constexpr int kVBlocksPerSM = 6;  // 33 KB of shared memory each
+constexpr int kSlotBytes = 8192;
 constexpr int kRing = 4;
+constexpr int kVecs = kSlotBytes / 16 / kVThreads;  // 16-byte vectors per thread per step
 constexpr int kMaxCluster = 16;
 
 // One value each CTA publishes to its cluster per exchange.
@@ -116,7 +118,8 @@ struct VerifyCta {
   int C, rank, tid, lane, warp;
   int lo, n;               // slice [lo, lo + n) of the vocabulary
   unsigned char* ring;     // kRing slots of kSlotBytes
-  uint64_t* bars;          // kRing mbarriers
+  uint64_t* bars;          // kRing "full" mbarriers (bytes landed)
+  uint64_t* empty;         // kRing "empty" mbarriers (one arrival per warp)
   Exch* ex;                // [2] published slots (double buffered)
   Exch* got;               // [kMaxCluster] gathered copies (read-only after a gather)
   float* red;              // [32] scratch
@@ -130,9 +133,16 @@ struct VerifyCta {
   // ---------------- streaming through the ring ----------------
   __device__ void issue(const T* src, uint32_t bytes) {
     const uint32_t r = issued % kRing;
+    const uint32_t use = issued / kRing;
+    if (threadIdx.x == 0 && !*(volatile int*)dead) {
+      // the slot's previous contents must have been read by every warp
+      if (use > 0 && !mbar_wait_bounded(smem_u32(&empty[r]), (use - 1) & 1u)) {
+        report_wait(st, kWhereVerifyLoad, request);
+        *(volatile int*)dead = 1;
+      }
+    }
     if (threadIdx.x == 0 && !*(volatile int*)dead) {
       const uint32_t b = smem_u32(&bars[r]);
-      // generic reads of the slot's previous contents are barrier-ordered before this
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(bytes)
                    : "memory");
@@ -144,6 +154,12 @@ struct VerifyCta {
     }
     ++issued;
   }
+  // every warp hands slot r back once it is done with it
+  __device__ void release(uint32_t r) {
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[r])) : "memory");
+  }
+  __device__ uint32_t slot_of(uint32_t k) const { return k % kRing; }
   __device__ const unsigned char* wait() {
     const uint32_t r = consumed % kRing;
     const uint32_t ph = (consumed / kRing) & 1u;
@@ -163,10 +179,13 @@ struct VerifyCta {
 
   // One pass over `nrow` (1 or 2) row slices, step by step; f(step, slot0,
   // slot1) runs in every thread once a step's slots have landed and must be
-  // done with them when it returns. f returns true to stop the pass early (the
-  // copies still in flight are drained).
+  // done with them when it returns. Fast passes (sync == false) run with no
+  // block barrier: warps move through the ring independently and hand slots
+  // back by arrivals. With sync == true every step is bracketed by block
+  // barriers and f may stop the pass early (returning true); the copies still
+  // in flight are then drained.
   template <class F>
-  __device__ void pass(const T* r0, const T* r1, int nrow, F f) {
+  __device__ void pass(const T* r0, const T* r1, int nrow, bool sync, F f) {
     const int ns = steps();
     const int ahead = kRing / nrow;
     int next = 0;
@@ -176,11 +195,15 @@ struct VerifyCta {
     }
     int s = 0;
     while (s < ns) {
+      const uint32_t ra = consumed % kRing;
       const unsigned char* a = wait();
+      const uint32_t rb = consumed % kRing;
       const unsigned char* b = (nrow == 2) ? wait() : nullptr;
-      __syncthreads();  // every thread sees the landed bytes and `dead`
+      if (sync) __syncthreads();
       const bool stop = f(s, a, b);
-      __syncthreads();  // the slots are free again
+      release(ra);
+      if (nrow == 2) release(rb);
+      if (sync) __syncthreads();
       ++s;
       if (stop) break;
       if (next < ns) {
@@ -190,15 +213,19 @@ struct VerifyCta {
       }
     }
     for (int k = s; k < next; ++k) {  // drain an early stop
-      wait();
-      if (nrow == 2) wait();
+      for (int q = 0; q < nrow; ++q) {
+        const uint32_t r = consumed % kRing;
+        wait();
+        release(r);
+      }
     }
     __syncthreads();
   }
 
-  // first element of this thread's vector h (0 or 1) of step s
-  __device__ __forceinline__ int vec_elem(int s, int h) const {
-    return s * kStepElems + (tid + h * kVThreads) * N;
+  // first element of this thread's vector m (0 .. kVecs-1) of step s; a step's
+  // vectors are in index order m * 128 + tid
+  __device__ __forceinline__ int vec_elem(int s, int m) const {
+    return s * kStepElems + (tid + m * kVThreads) * N;
   }
 
   // Publishes this CTA's value and gathers every CTA's (one cluster barrier).
@@ -241,29 +268,37 @@ struct VerifyCta {
   // CTA-wide online (max, sum 2^(z - max)) of z = v * cs over the slice of `row`.
   __device__ float2 row_stats(const T* row, float cs) {
     float m = -INFINITY, sum = 0.f;
-    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
+    pass(row, nullptr, 1, false, [&](int s, const unsigned char* a, const unsigned char*) {
+      float v[kVecs][N];
+      float vm = -INFINITY;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (vec_elem(s, h) >= n) continue;
-        float v[N];
-        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, v);
-        float vm = v[0];
+      for (int q = 0; q < kVecs; ++q) {
+        if (vec_elem(s, q) < n) {
+          Vec16<DT>::load(a + (tid + q * kVThreads) * 16, v[q]);
+        } else {
 #pragma unroll
-        for (int j = 1; j < N; ++j) vm = max_nan(vm, v[j]);
-        const float zm = vm * cs;
-        if (zm != zm) {  // NaN in this vector
-          sum = NAN;
-          continue;
+          for (int j = 0; j < N; ++j) v[q][j] = -INFINITY;
         }
-        if (zm > m) {
-          sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
-          m = zm;
-        }
-        if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
-          const float neg = -m;
 #pragma unroll
-          for (int j = 0; j < N; ++j) sum += ex2(fmaf(v[j], cs, neg));
-        }
+        for (int j = 0; j < N; ++j) vm = max_nan(vm, v[q][j]);
+      }
+      const float zm = vm * cs;
+      if (zm != zm) {  // a NaN in this step
+        sum = NAN;
+        return false;
+      }
+      if (zm > m) {
+        sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
+        m = zm;
+      }
+      if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
+        const float neg = -m;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < kVecs; ++q)
+#pragma unroll
+          for (int j = 0; j < N; ++j) acc[j & 3] += ex2(fmaf(v[q][j], cs, neg));
+        sum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
       }
       return false;
     });
@@ -275,13 +310,13 @@ struct VerifyCta {
     mv = -INFINITY;
     mi = 0x7fffffff;
     chk = -INFINITY;
-    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
+    pass(row, nullptr, 1, false, [&](int s, const unsigned char* a, const unsigned char*) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int e0 = vec_elem(s, h);
+      for (int q = 0; q < kVecs; ++q) {
+        const int e0 = vec_elem(s, q);
         if (e0 >= n) continue;
         float v[N];
-        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, v);
+        Vec16<DT>::load(a + (tid + q * kVThreads) * 16, v);
 #pragma unroll
         for (int j = 0; j < N; ++j) {
           chk = max_nan(chk, v[j]);
@@ -324,46 +359,49 @@ struct VerifyCta {
     int lastp = -1;  // last element of positive weight this thread has seen
     if (tid == 0) sint[0] = -1;
     __syncthreads();
-    pass(r0, r1, nrow, [&](int s, const unsigned char* a, const unsigned char* b) {
-      float vs[2], w[2][N];
+    pass(r0, r1, nrow, true, [&](int s, const unsigned char* a, const unsigned char* b) {
+      // this thread's vectors of the step are vectors q * 128 + tid in index order
+      float vs[kVecs], w[kVecs][N];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        vs[h] = 0.f;
+      for (int q = 0; q < kVecs; ++q) {
+        vs[q] = 0.f;
 #pragma unroll
-        for (int j = 0; j < N; ++j) w[h][j] = 0.f;
-        const int e0 = vec_elem(s, h);
+        for (int j = 0; j < N; ++j) w[q][j] = 0.f;
+        const int e0 = vec_elem(s, q);
         if (e0 >= n) continue;
         float tv[N], dv[N];
-        Vec16<DT>::load(a + (tid + h * kVThreads) * 16, tv);
-        if (b) Vec16<DT>::load(b + (tid + h * kVThreads) * 16, dv);
+        Vec16<DT>::load(a + (tid + q * kVThreads) * 16, tv);
+        if (b) Vec16<DT>::load(b + (tid + q * kVThreads) * 16, dv);
 #pragma unroll
         for (int j = 0; j < N; ++j) {
-          w[h][j] = wfun(tv[j], b ? dv[j] : 0.f);
-          vs[h] += w[h][j];
-          if (w[h][j] > 0.f) lastp = e0 + j;
+          w[q][j] = wfun(tv[j], b ? dv[j] : 0.f);
+          vs[q] += w[q][j];
+          if (w[q][j] > 0.f) lastp = e0 + j;
         }
       }
-      // exclusive prefix of the vectors' sums over the step (vector k = h * 128 + tid)
-      float pre[2];
+      // exclusive prefix of the vectors' sums over the step: red[q * 4 + warp]
+      // holds the warp totals in index order
+      float pre[kVecs];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float incl = warp_inclusive_scan(vs[h]);
-        if (lane == 31) red[h * 4 + warp] = incl;
-        pre[h] = incl - vs[h];
+      for (int q = 0; q < kVecs; ++q) {
+        const float incl = warp_inclusive_scan(vs[q]);
+        if (lane == 31) red[q * 4 + warp] = incl;
+        pre[q] = incl - vs[q];
       }
       __syncthreads();
-      float base[2], tot = 0.f, half0 = 0.f;
-      base[0] = pre[0];
-      base[1] = pre[1];
-      for (int k = 0; k < 4; ++k) {
-        half0 += red[k];
-        if (k < warp) {
-          base[0] += red[k];
-          base[1] += red[4 + k];
+      float base[kVecs], tot = 0.f;
+      {
+        float run = 0.f;
+#pragma unroll
+        for (int q = 0; q < kVecs; ++q) {
+          float before = run;
+          for (int k = 0; k < warp; ++k) before += red[q * 4 + k];
+          base[q] = before + pre[q];
+          for (int k = 0; k < 4; ++k) run += red[q * 4 + k];
         }
+        tot = run;
       }
-      base[1] += half0;
-      for (int k = 0; k < 8; ++k) tot += red[k];
+      __syncthreads();  // red is free again
       if (!(rem < tot)) {
         rem -= tot;
         return false;
@@ -372,22 +410,27 @@ struct VerifyCta {
       if (tid == 0) sint[1] = 0x7fffffff;
       __syncthreads();
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-        if (vs[h] > 0.f && rem < base[h] + vs[h]) atomicMin(&sint[1], h * kVThreads + tid);
+      for (int q = 0; q < kVecs; ++q)
+        if (vs[q] > 0.f && rem < base[q] + vs[q]) atomicMin(&sint[1], q * kVThreads + tid);
       __syncthreads();
       const int kv = sint[1];
       if (kv != 0x7fffffff && (kv % kVThreads) == tid) {
-        const int h = kv / kVThreads;
-        float r2 = rem - base[h];
+        const int qq = kv / kVThreads;
+        float r2 = 0.f;
         int f = -1, lp = -1;
 #pragma unroll
-        for (int j = 0; j < N; ++j) {
-          if (w[h][j] > 0.f) lp = j;
-          if (f < 0 && r2 < w[h][j]) f = j;
-          if (f < 0) r2 -= w[h][j];
+        for (int q = 0; q < kVecs; ++q) {
+          if (q != qq) continue;
+          r2 = rem - base[q];
+#pragma unroll
+          for (int j = 0; j < N; ++j) {
+            if (w[q][j] > 0.f) lp = j;
+            if (f < 0 && r2 < w[q][j]) f = j;
+            if (f < 0) r2 -= w[q][j];
+          }
         }
         if (f < 0) f = lp;
-        sint[0] = vec_elem(s, h) + max(f, 0);
+        sint[0] = vec_elem(s, qq) + max(f, 0);
       }
       __syncthreads();
       found = sint[0];
@@ -424,6 +467,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   using T = typename E::T;
   __shared__ __align__(128) unsigned char ring[kRing * kSlotBytes];
   __shared__ __align__(8) uint64_t bars[kRing];
+  __shared__ __align__(8) uint64_t empty[kRing];
   __shared__ Exch ex[2];
   __shared__ Exch got[kMaxCluster];
   __shared__ float rw[kMaxCluster];
@@ -439,6 +483,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   c.warp = c.tid >> 5;
   c.ring = ring;
   c.bars = bars;
+  c.empty = empty;
   c.ex = ex;
   c.got = got;
   c.red = red;
@@ -457,8 +502,11 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
 
   if (tid == 0) {
     dead = 0;
-    for (int i = 0; i < kRing; ++i)
+    for (int i = 0; i < kRing; ++i) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(&empty[i])), "r"(kVThreads / 32)
+                   : "memory");
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -581,14 +629,14 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
       return fmaxf(0.f, pp - qq);
     };
     float sr = 0.f;
-    c.pass(trow, drow, 2, [&](int s, const unsigned char* ta, const unsigned char* da) {
+    c.pass(trow, drow, 2, false, [&](int s, const unsigned char* ta, const unsigned char* da) {
       constexpr int N = Vec16<DT>::N;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (c.vec_elem(s, h) >= c.n) continue;
+      for (int q = 0; q < kVecs; ++q) {
+        if (c.vec_elem(s, q) >= c.n) continue;
         float tv[N], dv[N];
-        Vec16<DT>::load(ta + (tid + h * kVThreads) * 16, tv);
-        Vec16<DT>::load(da + (tid + h * kVThreads) * 16, dv);
+        Vec16<DT>::load(ta + (tid + q * kVThreads) * 16, tv);
+        Vec16<DT>::load(da + (tid + q * kVThreads) * 16, dv);
 #pragma unroll
         for (int j = 0; j < N; ++j) sr += resid(tv[j], dv[j]);
       }
@@ -635,11 +683,13 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
 
 int verify_cluster_size(int B, int V, int dtype, int num_sms) {
   // Enough CTAs in flight to keep HBM busy (kVBlocksPerSM 128-thread CTAs per
-  // SM), at most 16 per request, and at least one ring step per CTA.
+  // SM), at most 16 per request, and at least one ring step per CTA; measured
+  // on B200 at B = 256, V = 129280: C = 4 (one wave) beats 2, 8 and 16.
   const int es = dtype == DSPARK_F32 ? 4 : 2;
   const long long slots = (long long)kVBlocksPerSM * num_sms;
+  // about one wave: B * C up to 1.2x the resident CTA slots
   int C = 1;
-  while (C < kMaxCluster && (long long)B * C * 2 <= slots &&
+  while (C < kMaxCluster && (long long)B * C * 2 * 5 <= slots * 6 &&
          (long long)V * es / (2 * C) >= kSlotBytes)
     C <<= 1;
   return C;
