@@ -48,58 +48,77 @@ def peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clocks and clock-event reasons sampled through NVML (read-only
+    queries) on a background thread during the timed region."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.stop_ev = threading.Event()
+        self.thread = None
         try:
+            import pynvml
+            pynvml.nvmlInit()
             u = str(torch.cuda.get_device_properties(device_index).uuid)
-            self.idx = u if u.startswith("GPU-") else "GPU-" + u
+            u = u if u.startswith("GPU-") else "GPU-" + u
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(u)
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+            self.thread = threading.Thread(target=self._run, daemon=True)
         except Exception:
-            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
-            self.idx = vis.split(",")[device_index] if vis else str(device_index)
-        self.proc = None
-        self.path = os.path.join("/tmp", f"dspark_clocks_{os.getpid()}.csv")
+            self.thread = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            except Exception:
+                pass
+            self.stop_ev.wait(self.period)
 
     def start(self):
-        try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+        if self.thread:
+            self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if not self.thread:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.f.close()
-        sm, mx, reasons = [], 0.0, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = max(mx, float(parts[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        os.unlink(self.path)
-        if not sm:
+        self.stop_ev.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
             return None
-        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(n for bit, n in self.REASONS.items() if self.reasons & bit),
+                "samples": len(self.samples), "source": "NVML every 2 ms over the timed region"}
+
+
+def profiled_traffic(kernel_file: str, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel's source changed after the counters were taken."""
+    import hashlib
+    src = os.path.join(ROOT, "speculative_decoding_draft_sample_b200", "csrc", kernel_file)
+    path = os.path.join(ROOT, "profiles", summary)
+    if not (os.path.exists(src) and os.path.exists(path)):
+        return None, "no ncu summary committed"
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    fields = {}
+    for line in open(path):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("source_sha256") != sha:
+        return None, "kernel source changed since the ncu capture"
+    try:
+        return float(fields["dram_bytes_per_launch"]), "profiles/" + summary
+    except (KeyError, ValueError):
+        return None, "no dram_bytes_per_launch line"
 
 
 def time_region(fn, stream, iters: int) -> float:
@@ -173,7 +192,7 @@ def reference_arm(args, w: wl.Workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -256,15 +275,26 @@ def main():
         ms_verify = time_region(lambda: bn.verify(
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
             round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream), stream, 20)
+
+        # the dominant kernel alone: the draft-logit kernel of positions 1..K,
+        # one launch each (x already holds this round's tokens, so every
+        # launch sees the same inputs as in the round)
+        def logits_all():
+            for k in range(1, w.K + 1):
+                bn.draft_logits(dev["base"], dev["U"], dev["W"], dev["bias_scale"],
+                                dev["last_tok"], rnd.x, dev["temp"], k, rnd.d, rnd.ws, stream)
+        logits_all()
+        ms_logits = time_region(logits_all, stream, 10) / w.K
     # verify's algorithmic bytes: target rows 0..a_b of every request, plus the
     # draft row a_b of every request rejected before its cut
     rej = int((acc_np < cut).sum())
     verify_bytes = (int((acc_np + 1).sum()) + rej) * w.V * s_bytes
     verify_gbs = verify_bytes / (ms_verify * 1e-3) / 1e9
-    # draft stage: base in + d out per position, W once per position
-    draft_bytes_pos = 2 * w.B * w.V * s_bytes + w.r * w.V * s_bytes
-    draft_gbs = w.K * draft_bytes_pos / (ms_draft * 1e-3) / 1e9
-    gemm_tflops = 2.0 * w.B * w.r * w.V * w.K / (ms_draft * 1e-3) / 1e12
+    # draft-logit kernel, per launch: the base block in, d out, W once
+    logits_bytes = 2 * w.B * w.V * s_bytes + w.r * w.V * s_bytes
+    logits_gbs = logits_bytes / (ms_logits * 1e-3) / 1e9
+    draft_gbs = w.K * logits_bytes / (ms_draft * 1e-3) / 1e9
+    gemm_tflops = 2.0 * w.B * w.r * w.V / (ms_logits * 1e-3) / 1e12
 
     # end to end through the public API from pinned host buffers
     host = to_device(inp, pin=True)
@@ -281,11 +311,13 @@ def main():
                                               stream=stream), stream, e2e_steps)
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
-    dominant = "verify" if ms_verify >= ms_draft / w.K else "draft"
-    roof = {"kernel": "verify_kernel (dspark_verify)", "bound": "hbm", "achieved": verify_gbs,
-            "peak": hbm, "unit": "GB/s", "frac": verify_gbs / hbm, "traffic": None,
-            "peak_source": f"hbm_gbs of {peak_kind} peaks", "bytes_per_launch": verify_bytes,
-            "launch_ms": ms_verify}
+    traffic, traffic_src = profiled_traffic("draft_tc.cu", "draft_logits_tc_dspark5.txt")
+    roof = {"kernel": "draft_logits_tc (dspark_draft_logits, one draft position)", "bound": "hbm",
+            "achieved": logits_gbs, "peak": hbm, "unit": "GB/s", "frac": logits_gbs / hbm,
+            "traffic": traffic, "traffic_source": traffic_src,
+            "peak_source": f"hbm_gbs of {peak_kind} peaks",
+            "bytes_per_launch": logits_bytes, "launch_ms": ms_logits,
+            "share_of_step": w.K * ms_logits / ms}
     line = {
         "metric": METRIC, "value": rounds_per_s, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -299,11 +331,12 @@ def main():
         "emitted_tok_per_s": emit_all * 1000.0 / ms,
         "accepted_per_round": accepted, "emitted_per_round": emitted,
         "mean_cut": float(cut.mean()), "mean_accepted": float(acc_np.mean()),
-        "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify},
-        "verify_gbs": verify_gbs, "verify_frac_of_peak": verify_gbs / hbm,
-        "draft_stage": {"gbs": draft_gbs, "bytes_per_position": draft_bytes_pos,
-                        "bias_gemm_tflops": gemm_tflops, "tflops_peak": tflops},
-        "dominant_stage": dominant,
+        "stages_ms": {"draft": ms_draft, "draft_logits_per_launch": ms_logits,
+                      "schedule": ms_sched, "verify": ms_verify},
+        "verify": {"gbs": verify_gbs, "frac_of_hbm_peak": verify_gbs / hbm,
+                   "bytes_per_launch": verify_bytes, "launch_ms": ms_verify},
+        "draft_stage": {"gbs": draft_gbs, "bias_gemm_tflops_per_launch": gemm_tflops,
+                        "bias_gemm_frac_of_bf16_peak": gemm_tflops / tflops},
         "roofline": roof,
         "e2e": {"value": world * 1000.0 / ms_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},

@@ -4,6 +4,8 @@
  *
  *   dspark_draft_sample    semi-autoregressive draft: parallel base logits plus
  *                          a low-rank Markov-head bias, sampled position by position
+ *                          (dspark_draft_logits / dspark_draft_pick: one position's
+ *                          two halves)
  *   dspark_prefix_schedule calibrated confidence, survival products and the
  *                          early-stopping prefix cut against a cost-per-token table
  *   dspark_verify          lossless rejection-sampling verification, residual or
@@ -119,6 +121,40 @@ int dspark_draft_sample(const void* base, const void* U, const void* W,
                         uint64_t seed, uint64_t round_id, int32_t* x, void* d,
                         float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
                         dspark_stream_t stream);
+
+/*
+ * The two halves of one draft position of dspark_draft_sample, for callers
+ * that interleave other work between positions or time the halves apart.
+ * Calling, for k = 1..K in turn, dspark_draft_logits(k) then
+ * dspark_draft_pick(k) on one stream with one workspace gives results
+ * identical to dspark_draft_sample (the same kernels run in the same order).
+ * [P1] "DSpark's semi-autoregressive compromise"; [P3] "The Semi-Autoregressive
+ * Trick".
+ *
+ * dspark_draft_logits(k): d[:, k-1, :] = round_dtype(base[:, k-1, :] +
+ *   bias_scale * U[x_{k-1}] @ W), with x_{b,0} = last_tok[b] and x_{b,k-1} =
+ *   x[b, k-2] for k >= 2 (so x[:, k-2] must hold position k-1's tokens), and
+ *   the per-(request, 256-entry chunk) softmax partials of d/temp, kept in the
+ *   workspace for the pick that follows. Arguments as for dspark_draft_sample.
+ * dspark_draft_pick(k): x[:, k-1], q_lse[:, k-1], q_tok[:, k-1] from
+ *   d[:, k-1, :] and the workspace partials that dspark_draft_logits(k) left
+ *   (the workspace must not be used by another call in between). last_tok is
+ *   read only to report a bad token at k = 1.
+ * Both need 1 <= k <= K and a workspace of
+ * dspark_workspace_bytes(DSPARK_OP_DRAFT, B, K, V, r, dtype) bytes (pick takes
+ * no r; the size does not depend on it). Errors as for dspark_draft_sample.
+ */
+int dspark_draft_logits(const void* base, const void* U, const void* W,
+                        const float* bias_scale, const int32_t* last_tok,
+                        const int32_t* x, const float* temp, int B, int K, int V,
+                        int r, int dtype, int k, void* d, void* ws, size_t ws_bytes,
+                        dspark_stream_t stream);
+
+int dspark_draft_pick(const void* d, const int32_t* last_tok, const float* temp,
+                      int B, int K, int V, int dtype, uint64_t seed,
+                      uint64_t round_id, int k, int32_t* x, float* q_lse,
+                      float* q_tok, void* ws, size_t ws_bytes,
+                      dspark_stream_t stream);
 
 /*
  * Calibrated confidence, survival and the prefix cut.

@@ -38,6 +38,10 @@ SIGNATURES = {
     "dspark_prefix_schedule": (_i, [_p, _p, _p, _f, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
                            _p, _sz, _p]),
+    "dspark_draft_logits": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p,
+                                 _sz, _p]),
+    "dspark_draft_pick": (_i, [_p, _p, _p, _i, _i, _i, _i, _u64, _u64, _i, _p, _p, _p, _p, _sz,
+                               _p]),
     "dspark_draft_sample_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
                                         _p, _p, _p, _p, _p, _p]),
     "dspark_read_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32),
@@ -122,6 +126,32 @@ def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: in
         _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream))
     _check(rc, "dspark_draft_sample")
+
+
+def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, stream=None) -> None:
+    """dspark_draft_logits: position k's draft logits d[:, k-1] and the chunk
+    partials (in ws) that dspark_draft_pick(k) reads."""
+    B, K, V = base.shape
+    r = U.shape[1]
+    dt = _dtype_code(base)
+    rc = lib().dspark_draft_logits(
+        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
+        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
+        _ptr(x, "x", torch.int32), _ptr(temp, "temp", torch.float32), B, K, V, r, dt, int(k),
+        _ptr(d, "d", base.dtype), _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "dspark_draft_logits")
+
+
+def draft_pick(d, last_tok, temp, seed: int, round_id: int, k: int, x, q_lse, q_tok, ws,
+               stream=None) -> None:
+    """dspark_draft_pick: position k's token, q_lse and q_tok from d[:, k-1]."""
+    B, K, V = d.shape
+    rc = lib().dspark_draft_pick(
+        _ptr(d, "d"), _ptr(last_tok, "last_tok", torch.int32), _ptr(temp, "temp", torch.float32),
+        B, K, V, _dtype_code(d), seed, round_id, int(k), _ptr(x, "x", torch.int32),
+        _ptr(q_lse, "q_lse", torch.float32), _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "dspark_draft_pick")
 
 
 def draft_sample_static(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: int,

@@ -94,22 +94,27 @@ int dspark_read_status(void* ws, dspark_stream_t stream, uint32_t* code, int32_t
   return dspark_clear_status(ws, stream);
 }
 
-int dspark_draft_sample(const void* base, const void* U, const void* W, const float* bias_scale,
-                        const int32_t* last_tok, const float* temp, int B, int K, int V, int r,
-                        int dtype, uint64_t seed, uint64_t round_id, int32_t* x, void* d,
-                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
-                        dspark_stream_t stream) {
-  if (!base || !U || !W || !last_tok || !temp || !x || !d || !q_lse || !q_tok || !ws)
-    return DSPARK_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Argument checks and DraftArgs of the draft entry points. `logits` / `pick`
+// select which of the two kernels the caller is about to launch; the pointers
+// only the other one reads may be null.
+int draft_prepare(DraftArgs& a, int* sms, bool logits, bool pick, const void* base, const void* U,
+                  const void* W, const float* bias_scale, const int32_t* last_tok, const float* temp,
+                  int B, int K, int V, int r, int dtype, uint64_t seed, uint64_t round_id, int32_t* x,
+                  void* d, float* q_lse, float* q_tok, void* ws, size_t ws_bytes) {
+  if (!last_tok || !temp || !x || !d || !ws) return DSPARK_ERR_INVALID_ARG;
+  if (logits && (!base || !U || !W)) return DSPARK_ERR_INVALID_ARG;
+  if (pick && (!q_lse || !q_tok)) return DSPARK_ERR_INVALID_ARG;
   if (!shape_ok(B, K, V, dtype) || r < 1 || r > 1024) return DSPARK_ERR_INVALID_ARG;
-  if (dtype == DSPARK_BF16 && r % 16 != 0) return DSPARK_ERR_UNSUPPORTED;
-  if (!aligned16(base) || !aligned16(U) || !aligned16(W) || !aligned16(d) || !aligned16(ws))
-    return DSPARK_ERR_INVALID_ARG;
+  if (logits && dtype == DSPARK_BF16 && r % 16 != 0) return DSPARK_ERR_UNSUPPORTED;
+  if (!aligned16(d) || !aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
+  if (logits && (!aligned16(base) || !aligned16(U) || !aligned16(W))) return DSPARK_ERR_INVALID_ARG;
   if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_DRAFT, B, K, V, r, dtype))
     return DSPARK_ERR_WORKSPACE;
-  int sms = 0;
-  if (int e = device_check(&sms)) return e;
-  DraftArgs a;
+  if (int e = device_check(sms)) return e;
   a.base = base;
   a.U = U;
   a.W = W;
@@ -130,14 +135,59 @@ int dspark_draft_sample(const void* base, const void* U, const void* W, const fl
   a.status = static_cast<Status*>(ws);
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   a.nchunk = nchunks(V);
+  return DSPARK_OK;
+}
+
+cudaError_t launch_logits(const DraftArgs& a, int k, int sms, cudaStream_t s) {
+  return draft_tc_supported(a) ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dspark_draft_sample(const void* base, const void* U, const void* W, const float* bias_scale,
+                        const int32_t* last_tok, const float* temp, int B, int K, int V, int r,
+                        int dtype, uint64_t seed, uint64_t round_id, int32_t* x, void* d,
+                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
+                        dspark_stream_t stream) {
+  DraftArgs a;
+  int sms = 0;
+  if (int e = draft_prepare(a, &sms, true, true, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
+                            dtype, seed, round_id, x, d, q_lse, q_tok, ws, ws_bytes))
+    return e;
   cudaStream_t s = (cudaStream_t)stream;
-  const bool tc = draft_tc_supported(a);
   for (int k = 1; k <= K; ++k) {
-    cudaError_t e = tc ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
+    cudaError_t e = launch_logits(a, k, sms, s);
     if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
     if (e != cudaSuccess) return DSPARK_ERR_CUDA;
   }
   return DSPARK_OK;
+}
+
+int dspark_draft_logits(const void* base, const void* U, const void* W, const float* bias_scale,
+                        const int32_t* last_tok, const int32_t* x, const float* temp, int B, int K,
+                        int V, int r, int dtype, int k, void* d, void* ws, size_t ws_bytes,
+                        dspark_stream_t stream) {
+  if (k < 1 || k > K) return DSPARK_ERR_INVALID_ARG;
+  DraftArgs a;
+  int sms = 0;
+  if (int e = draft_prepare(a, &sms, true, false, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
+                            dtype, 0, 0, const_cast<int32_t*>(x), d, nullptr, nullptr, ws, ws_bytes))
+    return e;
+  return cuda_status(launch_logits(a, k, sms, (cudaStream_t)stream));
+}
+
+int dspark_draft_pick(const void* d, const int32_t* last_tok, const float* temp, int B, int K, int V,
+                      int dtype, uint64_t seed, uint64_t round_id, int k, int32_t* x, float* q_lse,
+                      float* q_tok, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (k < 1 || k > K) return DSPARK_ERR_INVALID_ARG;
+  DraftArgs a;
+  if (int e = draft_prepare(a, nullptr, false, true, nullptr, nullptr, nullptr, nullptr, last_tok, temp,
+                            B, K, V, 16, dtype, seed, round_id, x, const_cast<void*>(d), q_lse, q_tok,
+                            ws, ws_bytes))
+    return e;
+  return cuda_status(draft_sample_launch(a, k, (cudaStream_t)stream));
 }
 
 int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp, const float* step_cost,

@@ -15,7 +15,9 @@
 //
 // Persistent CTAs, one per SM, warp-specialised:
 //   warp 0     TMA producer of W tiles (ring of four 16 KB stages of 32 ranks)
-//   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer
+//   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer (it
+//              waits at a named barrier for A, which the epilogue warps gather
+//              while the producers already stream W and base)
 //   warp 2     TMA producer of base tiles (ring of six 16 KB [128 x 64] blocks,
 //              so the next tile's blocks load while this one is processed)
 //   warps 4-11 epilogue, two halves of four warps (one per TMEM lane
@@ -149,6 +151,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// Named barrier 4: the eight epilogue warps arrive once A is in shared memory,
+// the MMA warp waits for them.
+__device__ __forceinline__ void a_ready_arrive() {
+  asm volatile("bar.arrive 4, 288;" ::: "memory");
+}
+__device__ __forceinline__ void a_ready_sync() {
+  asm volatile("bar.sync 4, 288;" ::: "memory");
+}
 __device__ __forceinline__ void half_bar(int h) {  // the four warps of one epilogue half
   asm volatile("bar.sync %0, 128;" ::"r"(1 + h) : "memory");
 }
@@ -242,26 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
 
-  // A = U[prev_b, :] for the 128 rows of this M-tile, 128-byte swizzled, K-major:
-  // k-block kb (64 ranks) at kb * 16 KB, row m at m * 128 B, 16-byte chunk c at
-  // (c ^ (m & 7)) * 16 B. Rows past B and ranks past r are zero.
-  {
-    const uint16_t* U = static_cast<const uint16_t*>(p.U);
-    const int chunks_per_row = 32;  // 256 ranks / 8
-    for (int e = tid; e < kTileM * chunks_per_row; e += kThreads) {
-      const int m = e / chunks_per_row, cc = e % chunks_per_row;
-      const int b = m0 + m;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (b < p.B && cc * 8 < p.r) {
-        int tok = p.prev[(long long)b * p.prev_stride];
-        if (tok < 0 || tok >= p.V) tok = 0;  // reported by the sampler
-        v = *reinterpret_cast<const uint4*>(U + (long long)tok * p.r + cc * 8);
-      }
-      const int kb = cc >> 3, c = cc & 7;
-      *reinterpret_cast<uint4*>(sA + kb * 16384 + m * 128 + ((c ^ (m & 7)) << 4)) = v;
-    }
-    fence_async_smem();
-  }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -317,8 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*(volatile int*)abort_flag)
       for (int q = 0; q < kBaseSlots; ++q)
         if (last[q] >= 0) mbar_wait(&b_full[q], (last[q] / kBaseSlots) & 1);
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // A is gathered by the epilogue warps meanwhile (the producers are already
+    // streaming W and base); the whole warp waits for it at the named barrier
+    a_ready_sync();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (lane == 0) {
     int it = 0;
     int last_it = -1;  // last W stage whose MMAs were committed
     const uint32_t a_base = su32(sA);
@@ -375,7 +370,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     // MMAs complete in order: once the last commit has landed, tensor memory is quiet
     if (*(volatile int*)abort_flag && last_it >= 0)
       mbar_wait(&w_empty[last_it % kWStages], (last_it / kWStages) & 1);
+    }
   } else if (warp >= 4) {
+    // ---------------- A gather, then the epilogue ----------------
+    // A = U[prev_b, :] for the 128 rows of this M-tile, 128-byte swizzled,
+    // K-major: k-block kb (64 ranks) at kb * 16 KB, row m at m * 128 B, 16-byte
+    // chunk c at (c ^ (m & 7)) * 16 B. Rows past B and ranks past r are zero.
+    // Epilogue warp e gathers rows 16e .. 16e + 15: lanes 0-15 read the rows'
+    // tokens, then every lane loads one 16-byte chunk of each of the 16 rows
+    // (all loads in flight at once; a row is one 512-byte coalesced read).
+    {
+      const int ew = warp - 4;
+      int tokv = 0;
+      if (lane < 16) {
+        const int b = m0 + ew * 16 + lane;
+        if (b < p.B) tokv = p.prev[(long long)b * p.prev_stride];
+        if (tokv < 0 || tokv >= p.V) tokv = 0;  // reported by the sampler
+      }
+      const uint16_t* U = static_cast<const uint16_t*>(p.U);
+      uint4 v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int tok = __shfl_sync(0xffffffffu, tokv, i);
+        v[i] = make_uint4(0, 0, 0, 0);
+        if (m0 + ew * 16 + i < p.B && lane * 8 < p.r)
+          v[i] = *reinterpret_cast<const uint4*>(U + (long long)tok * p.r + lane * 8);
+      }
+      const int kb = lane >> 3, c = lane & 7;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int m = ew * 16 + i;
+        *reinterpret_cast<uint4*>(sA + kb * 16384 + m * 128 + ((c ^ (m & 7)) << 4)) = v[i];
+      }
+      fence_async_smem();
+      a_ready_arrive();
+    }
     // ---------------- epilogue ----------------
     const int q = warp & 3;             // TMEM lane quadrant
     const int h = (warp - 4) >> 2;      // half: column blocks h and h + 2

@@ -16,20 +16,26 @@
 // through a ring of 8 KB shared-memory slots filled by bulk asynchronous copies
 // (cp.async.bulk; a "full" mbarrier per slot completes with the bytes, a
 // per-warp "empty" arrival hands the slot back): no row is kept resident, so a
-// CTA needs 33 KB of shared memory and every request of the batch is in flight
+// CTA needs 35 KB of shared memory and every request of the batch is in flight
 // at once. One online (max, sum 2^z) pass per row and one exchange over
-// distributed shared memory give the row's normaliser; only the CTA that owns
-// an inverse-CDF crossing streams its slice again (from L2) to place the token.
+// distributed shared memory give the row's normaliser. Every pass also leaves
+// per-step, per-warp partial sums ("records"), so an inverse-CDF placement
+// rescans one 8 KB step of one CTA (from L2) instead of its whole slice.
+#include <algorithm>
+
 #include "common.cuh"
 #include "verify.cuh"
 
 namespace dspark {
 
 constexpr int kVThreads = 128;
-constexpr int kVBlocksPerSM = 6;  // 33 KB of shared memory each
+constexpr int kVWarps = kVThreads / 32;
+constexpr int kVBlocksPerSM = 6;  // 35 KB of shared memory each
 constexpr int kSlotBytes = 8192;
 constexpr int kRing = 4;
-constexpr int kVecs = kSlotBytes / 16 / kVThreads;  // 16-byte vectors per thread per step
+constexpr int kThreadBytes = kSlotBytes / kVThreads;  // contiguous bytes per thread per step
+constexpr int kVecs = kThreadBytes / 16;              // 16-byte vectors per thread per step
+constexpr int kMaxRec = 64;                           // placement records per CTA
 constexpr int kMaxCluster = 16;
 
 // One value each CTA publishes to its cluster per exchange.
@@ -108,20 +114,30 @@ __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float
   m = mm;
 }
 
+// NaN-propagating maximum over a warp.
+__device__ __forceinline__ float warp_max_nan(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = max_nan(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
 template <int DT>
 struct VerifyCta {
   using E = Elem<DT>;
   using T = typename E::T;
-  static constexpr int N = Vec16<DT>::N;            // elements per 16-byte vector
+  static constexpr int N = Vec16<DT>::N;                    // elements per 16-byte vector
   static constexpr int kStepElems = kSlotBytes / E::kBytes;
+  static constexpr int kThreadElems = kThreadBytes / E::kBytes;
 
   int C, rank, tid, lane, warp;
   int lo, n;               // slice [lo, lo + n) of the vocabulary
+  int G, nrec;             // ring steps per record, records in use
   unsigned char* ring;     // kRing slots of kSlotBytes
   uint64_t* bars;          // kRing "full" mbarriers (bytes landed)
   uint64_t* empty;         // kRing "empty" mbarriers (one arrival per warp)
   Exch* ex;                // [2] published slots (double buffered)
   Exch* got;               // [kMaxCluster] gathered copies (read-only after a gather)
+  float2* rec;             // [kMaxRec][kVWarps] per record and warp: (reference max, sum)
   float* red;              // [32] scratch
   int* sint;               // [4] scratch
   int* dead;               // set once a wait gave up
@@ -159,7 +175,6 @@ struct VerifyCta {
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&empty[r])) : "memory");
   }
-  __device__ uint32_t slot_of(uint32_t k) const { return k % kRing; }
   __device__ const unsigned char* wait() {
     const uint32_t r = consumed % kRing;
     const uint32_t ph = (consumed / kRing) & 1u;
@@ -176,16 +191,14 @@ struct VerifyCta {
   __device__ uint32_t step_bytes(int s) const {
     return (uint32_t)min(kStepElems, n - s * kStepElems) * E::kBytes;
   }
+  __device__ bool record_end(int s) const { return (s + 1) % G == 0 || s + 1 == steps(); }
 
-  // One pass over `nrow` (1 or 2) row slices, step by step; f(step, slot0,
-  // slot1) runs in every thread once a step's slots have landed and must be
-  // done with them when it returns. Fast passes (sync == false) run with no
-  // block barrier: warps move through the ring independently and hand slots
-  // back by arrivals. With sync == true every step is bracketed by block
-  // barriers and f may stop the pass early (returning true); the copies still
-  // in flight are then drained.
+  // One pass over `nrow` (1 or 2) row slices, step by step, with no block
+  // barrier inside: warps move through the ring independently and hand slots
+  // back by arrivals. f(step, slot0, slot1) runs in every thread once the
+  // step's slots have landed and must be done with them when it returns.
   template <class F>
-  __device__ void pass(const T* r0, const T* r1, int nrow, bool sync, F f) {
+  __device__ void pass(const T* r0, const T* r1, int nrow, F f) {
     const int ns = steps();
     const int ahead = kRing / nrow;
     int next = 0;
@@ -193,39 +206,33 @@ struct VerifyCta {
       issue(r0 + next * kStepElems, step_bytes(next));
       if (nrow == 2) issue(r1 + next * kStepElems, step_bytes(next));
     }
-    int s = 0;
-    while (s < ns) {
+    for (int s = 0; s < ns; ++s) {
       const uint32_t ra = consumed % kRing;
       const unsigned char* a = wait();
       const uint32_t rb = consumed % kRing;
       const unsigned char* b = (nrow == 2) ? wait() : nullptr;
-      if (sync) __syncthreads();
-      const bool stop = f(s, a, b);
+      f(s, a, b);
       release(ra);
       if (nrow == 2) release(rb);
-      if (sync) __syncthreads();
-      ++s;
-      if (stop) break;
       if (next < ns) {
         issue(r0 + next * kStepElems, step_bytes(next));
         if (nrow == 2) issue(r1 + next * kStepElems, step_bytes(next));
         ++next;
       }
     }
-    for (int k = s; k < next; ++k) {  // drain an early stop
-      for (int q = 0; q < nrow; ++q) {
-        const uint32_t r = consumed % kRing;
-        wait();
-        release(r);
-      }
-    }
     __syncthreads();
   }
 
-  // first element of this thread's vector m (0 .. kVecs-1) of step s; a step's
-  // vectors are in index order m * 128 + tid
-  __device__ __forceinline__ int vec_elem(int s, int m) const {
-    return s * kStepElems + (tid + m * kVThreads) * N;
+  // A step gives thread t the 64 contiguous bytes [64 t, 64 t + 64) of its
+  // slot. The thread reads its four 16-byte vectors in the rotated order
+  // q ^ ((t >> 1) & 3), which spreads every 8-thread phase of a 128-bit
+  // shared-memory load over all 32 banks.
+  __device__ __forceinline__ int rot(int q) const { return q ^ ((tid >> 1) & 3); }
+  __device__ __forceinline__ int vec_elem(int s, int q) const {
+    return s * kStepElems + tid * kThreadElems + rot(q) * N;
+  }
+  __device__ __forceinline__ const unsigned char* vec_ptr(const unsigned char* slot, int q) const {
+    return slot + tid * kThreadBytes + (rot(q) << 4);
   }
 
   // Publishes this CTA's value and gathers every CTA's (one cluster barrier).
@@ -251,7 +258,7 @@ struct VerifyCta {
     }
     __syncthreads();
     float M = red[0], S = red[8];
-    for (int w = 1; w < kVThreads / 32; ++w) online_merge(M, S, red[w], red[8 + w]);
+    for (int w = 1; w < kVWarps; ++w) online_merge(M, S, red[w], red[8 + w]);
     __syncthreads();
     return make_float2(M, S);
   }
@@ -260,21 +267,23 @@ struct VerifyCta {
     if (lane == 0) red[warp] = v;
     __syncthreads();
     float t = 0.f;
-    for (int w = 0; w < kVThreads / 32; ++w) t += red[w];
+    for (int w = 0; w < kVWarps; ++w) t += red[w];
     __syncthreads();
     return t;
   }
 
-  // CTA-wide online (max, sum 2^(z - max)) of z = v * cs over the slice of `row`.
+  // CTA-wide online (max, sum 2^(z - max)) of z = v * cs over the slice of
+  // `row`. The reference maximum moves per warp and step (warp-uniform), and
+  // every record keeps its warp's (maximum, sum) for a later placement.
   __device__ float2 row_stats(const T* row, float cs) {
-    float m = -INFINITY, sum = 0.f;
-    pass(row, nullptr, 1, false, [&](int s, const unsigned char* a, const unsigned char*) {
+    float m = -INFINITY, sum = 0.f, rs = 0.f;
+    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
       float v[kVecs][N];
       float vm = -INFINITY;
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
         if (vec_elem(s, q) < n) {
-          Vec16<DT>::load(a + (tid + q * kVThreads) * 16, v[q]);
+          Vec16<DT>::load(vec_ptr(a, q), v[q]);
         } else {
 #pragma unroll
           for (int j = 0; j < N; ++j) v[q][j] = -INFINITY;
@@ -282,25 +291,34 @@ struct VerifyCta {
 #pragma unroll
         for (int j = 0; j < N; ++j) vm = max_nan(vm, v[q][j]);
       }
-      const float zm = vm * cs;
-      if (zm != zm) {  // a NaN in this step
+      const float zm = warp_max_nan(vm) * cs;
+      if (zm != zm) {  // a NaN in this step: the sums stay NaN from here on
         sum = NAN;
-        return false;
-      }
-      if (zm > m) {
-        sum = (m == -INFINITY) ? sum : sum * ex2(m - zm);
-        m = zm;
-      }
-      if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
-        const float neg = -m;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        rs = NAN;
+      } else {
+        if (zm > m) {
+          const float sc = (m == -INFINITY) ? 0.f : ex2(m - zm);
+          sum *= sc;
+          rs *= sc;
+          m = zm;
+        }
+        if (m != -INFINITY) {  // entries at -inf weigh nothing; +inf makes the sum NaN
+          const float neg = -m;
+          float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int q = 0; q < kVecs; ++q)
+          for (int q = 0; q < kVecs; ++q)
 #pragma unroll
-          for (int j = 0; j < N; ++j) acc[j & 3] += ex2(fmaf(v[q][j], cs, neg));
-        sum += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            for (int j = 0; j < N; ++j) acc[j & 3] += ex2(fmaf(v[q][j], cs, neg));
+          const float t = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+          sum += t;
+          rs += t;
+        }
       }
-      return false;
+      if (record_end(s)) {
+        const float t = warp_sum(rs);
+        if (lane == 0) rec[(s / G) * kVWarps + warp] = make_float2(m, t);
+        rs = 0.f;
+      }
     });
     return block_online(m, sum);
   }
@@ -310,30 +328,31 @@ struct VerifyCta {
     mv = -INFINITY;
     mi = 0x7fffffff;
     chk = -INFINITY;
-    pass(row, nullptr, 1, false, [&](int s, const unsigned char* a, const unsigned char*) {
+    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
         const int e0 = vec_elem(s, q);
         if (e0 >= n) continue;
         float v[N];
-        Vec16<DT>::load(a + (tid + q * kVThreads) * 16, v);
+        Vec16<DT>::load(vec_ptr(a, q), v);
 #pragma unroll
         for (int j = 0; j < N; ++j) {
           chk = max_nan(chk, v[j]);
           argmax_merge(mv, mi, v[j], lo + e0 + j);
         }
       }
-      return false;
     });
   }
 
-  // Inverse-CDF placement of `thr` on the weights wfun(t_value, d_value) of the
-  // cluster's slices, in index order. rw[r] are the per-rank totals (identical
-  // in every CTA). Only the owning CTA streams its slice again; it returns the
-  // token in every thread, the other CTAs return -1, and -2 means that no rank
-  // holds positive mass. No cluster exchange happens here.
-  template <class F>
-  __device__ int place(float thr, const float* rw, const T* r0, const T* r1, int nrow, F wfun) {
+  // Inverse-CDF placement of `thr` on the weights wfun(t_value, d_value) of
+  // the cluster's slices, in index order. rw[r] are the per-rank totals
+  // (identical in every CTA). The owning CTA finds the record holding the
+  // crossing from the last pass's records (recw gives a record's weight), then
+  // rescans only that record's steps, straight from global memory. It returns
+  // the token in every thread; the other CTAs return -1, and -2 means that no
+  // rank holds positive mass. No cluster exchange happens here.
+  template <class F, class R>
+  __device__ int place(float thr, const float* rw, const T* r0, const T* r1, F wfun, R recw) {
     int owner = -1, lastpos = -1;
     float P = 0.f, Pown = 0.f;
     for (int r = 0; r < C; ++r) {
@@ -355,88 +374,75 @@ struct VerifyCta {
     if (owner < 0) return -2;
     if (owner != rank) return -1;
     float rem = fallback ? INFINITY : thr - Pown;
-    int found = -1;
-    int lastp = -1;  // last element of positive weight this thread has seen
-    if (tid == 0) sint[0] = -1;
-    __syncthreads();
-    pass(r0, r1, nrow, true, [&](int s, const unsigned char* a, const unsigned char* b) {
-      // this thread's vectors of the step are vectors q * 128 + tid in index order
-      float vs[kVecs], w[kVecs][N];
+    // the record holding the crossing (the same walk in every thread)
+    int g0 = -1, glast = -1;
+    for (int g = 0; g < nrec; ++g) {
+      float wg = 0.f;
+      for (int w = 0; w < kVWarps; ++w) wg += recw(rec[g * kVWarps + w]);
+      if (wg > 0.f) {
+        glast = g;
+        if (g0 < 0 && rem < wg) g0 = g;
+      }
+      if (g0 < 0) rem -= wg;
+    }
+    if (g0 < 0) {  // rounding: past the last record; its last positive element
+      g0 = max(glast, 0);
+      rem = INFINITY;
+    }
+    // rescan the record's steps: thread t weighs its kThreadElems contiguous
+    // elements of each step in index order
+    const int s_end = min(steps(), (g0 + 1) * G);
+    int found = -1, lastp = -1;
+    for (int s = g0 * G; s < s_end && found < 0; ++s) {
+      const int e0 = s * kStepElems + tid * kThreadElems;
+      float w[kThreadElems];
+      float ts = 0.f;
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
-        vs[q] = 0.f;
-#pragma unroll
-        for (int j = 0; j < N; ++j) w[q][j] = 0.f;
-        const int e0 = vec_elem(s, q);
-        if (e0 >= n) continue;
         float tv[N], dv[N];
-        Vec16<DT>::load(a + (tid + q * kVThreads) * 16, tv);
-        if (b) Vec16<DT>::load(b + (tid + q * kVThreads) * 16, dv);
+        const bool ok = e0 + q * N < n;
+        if (ok) {
+          Vec16<DT>::load(r0 + e0 + q * N, tv);
+          if (r1) Vec16<DT>::load(r1 + e0 + q * N, dv);
+        }
 #pragma unroll
         for (int j = 0; j < N; ++j) {
-          w[q][j] = wfun(tv[j], b ? dv[j] : 0.f);
-          vs[q] += w[q][j];
-          if (w[q][j] > 0.f) lastp = e0 + j;
+          w[q * N + j] = ok ? wfun(tv[j], r1 ? dv[j] : 0.f) : 0.f;
+          ts += w[q * N + j];
+          if (w[q * N + j] > 0.f) lastp = e0 + q * N + j;
         }
       }
-      // exclusive prefix of the vectors' sums over the step: red[q * 4 + warp]
-      // holds the warp totals in index order
-      float pre[kVecs];
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q) {
-        const float incl = warp_inclusive_scan(vs[q]);
-        if (lane == 31) red[q * 4 + warp] = incl;
-        pre[q] = incl - vs[q];
-      }
-      __syncthreads();
-      float base[kVecs], tot = 0.f;
-      {
-        float run = 0.f;
-#pragma unroll
-        for (int q = 0; q < kVecs; ++q) {
-          float before = run;
-          for (int k = 0; k < warp; ++k) before += red[q * 4 + k];
-          base[q] = before + pre[q];
-          for (int k = 0; k < 4; ++k) run += red[q * 4 + k];
-        }
-        tot = run;
-      }
-      __syncthreads();  // red is free again
-      if (!(rem < tot)) {
-        rem -= tot;
-        return false;
-      }
-      // the crossing is in this step: the first vector whose range holds it
+      // exclusive prefix of the thread sums over the step (thread order is index order)
+      const float incl_w = warp_inclusive_scan(ts);
+      if (lane == 31) red[warp] = incl_w;
       if (tid == 0) sint[1] = 0x7fffffff;
       __syncthreads();
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q)
-        if (vs[q] > 0.f && rem < base[q] + vs[q]) atomicMin(&sint[1], q * kVThreads + tid);
-      __syncthreads();
-      const int kv = sint[1];
-      if (kv != 0x7fffffff && (kv % kVThreads) == tid) {
-        const int qq = kv / kVThreads;
-        float r2 = 0.f;
-        int f = -1, lp = -1;
-#pragma unroll
-        for (int q = 0; q < kVecs; ++q) {
-          if (q != qq) continue;
-          r2 = rem - base[q];
-#pragma unroll
-          for (int j = 0; j < N; ++j) {
-            if (w[q][j] > 0.f) lp = j;
-            if (f < 0 && r2 < w[q][j]) f = j;
-            if (f < 0) r2 -= w[q][j];
-          }
-        }
-        if (f < 0) f = lp;
-        sint[0] = vec_elem(s, qq) + max(f, 0);
+      float excl = incl_w - ts, tot = 0.f;
+      for (int k = 0; k < kVWarps; ++k) {
+        if (k < warp) excl += red[k];
+        tot += red[k];
       }
+      if (rem < tot && ts > 0.f && rem < excl + ts) atomicMin(&sint[1], tid);
       __syncthreads();
-      found = sint[0];
-      if (found < 0) rem -= tot;  // rounding: no vector held it; the fallback below decides
-      return found >= 0;
-    });
+      const int kt = sint[1];
+      if (rem < tot && kt != 0x7fffffff) {
+        if (tid == kt) {
+          float r2 = rem - excl;
+          int f = -1, lp = -1;
+#pragma unroll
+          for (int j = 0; j < kThreadElems; ++j) {
+            if (w[j] > 0.f) lp = j;
+            if (f < 0 && w[j] > 0.f && r2 < w[j]) f = j;
+            if (f < 0) r2 -= w[j];
+          }
+          sint[0] = e0 + (f < 0 ? lp : f);
+        }
+        __syncthreads();
+        found = sint[0];
+      }
+      if (found < 0) rem -= tot;
+      __syncthreads();  // red and sint are free again
+    }
     if (found < 0) {  // no crossing (rounding only): the last element of positive weight
       if (tid == 0) sint[2] = -1;
       __syncthreads();
@@ -471,6 +477,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   __shared__ Exch ex[2];
   __shared__ Exch got[kMaxCluster];
   __shared__ float rw[kMaxCluster];
+  __shared__ float2 rec[kMaxRec * kVWarps];
   __shared__ float red[32];
   __shared__ int sint[4];
   __shared__ int dead;
@@ -486,6 +493,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   c.empty = empty;
   c.ex = ex;
   c.got = got;
+  c.rec = rec;
   c.red = red;
   c.sint = sint;
   c.dead = &dead;
@@ -497,6 +505,8 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   c.request = b;
   c.lo = c.rank * a.slice;
   c.n = max(0, min(a.slice, a.V - c.lo));
+  c.G = max(1, (c.steps() + kMaxRec - 1) / kMaxRec);
+  c.nrec = (c.steps() + c.G - 1) / c.G;
   Status* st = a.status;
   const int tid = c.tid;
 
@@ -601,8 +611,9 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
     }
     if (j == L) {  // every verified draft accepted: bonus token from p of row L
       const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kBonus);
-      y = c.place(u * Z, rw, row + c.lo, nullptr, 1,
-                  [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); });
+      y = c.place(u * Z, rw, row + c.lo, nullptr,
+                  [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); },
+                  [&](float2 r) { return r.x == -INFINITY ? 0.f : r.y * ex2(r.x - M); });
       break;
     }
     const float p = ex2(gtx - M) / Z;
@@ -628,19 +639,26 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
       const float qq = ex2(fmaf(dv, cs, -Mq)) * iZq;
       return fmaxf(0.f, pp - qq);
     };
-    float sr = 0.f;
-    c.pass(trow, drow, 2, false, [&](int s, const unsigned char* ta, const unsigned char* da) {
+    float sr = 0.f, rs = 0.f;
+    c.pass(trow, drow, 2, [&](int s, const unsigned char* ta, const unsigned char* da) {
       constexpr int N = Vec16<DT>::N;
+      float acc[2] = {0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
         if (c.vec_elem(s, q) >= c.n) continue;
         float tv[N], dv[N];
-        Vec16<DT>::load(ta + (tid + q * kVThreads) * 16, tv);
-        Vec16<DT>::load(da + (tid + q * kVThreads) * 16, dv);
+        Vec16<DT>::load(c.vec_ptr(ta, q), tv);
+        Vec16<DT>::load(c.vec_ptr(da, q), dv);
 #pragma unroll
-        for (int j = 0; j < N; ++j) sr += resid(tv[j], dv[j]);
+        for (int j = 0; j < N; ++j) acc[j & 1] += resid(tv[j], dv[j]);
       }
-      return false;
+      sr += acc[0] + acc[1];
+      rs += acc[0] + acc[1];
+      if (c.record_end(s)) {
+        const float t = warp_sum(rs);
+        if (c.lane == 0) rec[(s / c.G) * kVWarps + c.warp] = make_float2(0.f, t);
+        rs = 0.f;
+      }
     });
     const float totr = c.block_sum(sr);
     c.gather(Exch{0.f, totr, 0.f, 0});
@@ -650,14 +668,15 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
     __syncthreads();
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kResidual);
     if (R > 0.f) {
-      y = c.place(u * R, rw, trow, drow, 2, resid);
+      y = c.place(u * R, rw, trow, drow, resid, [](float2 r) { return r.y; });
     } else {
       // exact-zero residual (floating point only): draw from p instead
       const float2 mz = c.row_stats(trow, cs);
       c.gather(Exch{mz.x, mz.y, 0.f, 0});
       if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
       __syncthreads();
-      y = c.place(u * Z, rw, trow, nullptr, 1, [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); });
+      y = c.place(u * Z, rw, trow, nullptr, [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); },
+                  [&](float2 r) { return r.x == -INFINITY ? 0.f : r.y * ex2(r.x - M); });
     }
   }
 
@@ -683,11 +702,11 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
 
 int verify_cluster_size(int B, int V, int dtype, int num_sms) {
   // Enough CTAs in flight to keep HBM busy (kVBlocksPerSM 128-thread CTAs per
-  // SM), at most 16 per request, and at least one ring step per CTA; measured
-  // on B200 at B = 256, V = 129280: C = 4 (one wave) beats 2, 8 and 16.
+  // SM), at most 16 per request, and at least one ring step per CTA. Measured
+  // on B200 at B = 256, V = 129280: C = 4 (about 1.15 waves) beats 3 (one
+  // wave), 2, 6, 8 and 16.
   const int es = dtype == DSPARK_F32 ? 4 : 2;
   const long long slots = (long long)kVBlocksPerSM * num_sms;
-  // about one wave: B * C up to 1.2x the resident CTA slots
   int C = 1;
   while (C < kMaxCluster && (long long)B * C * 2 * 5 <= slots * 6 &&
          (long long)V * es / (2 * C) >= kSlotBytes)

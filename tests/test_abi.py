@@ -52,6 +52,8 @@ def test_null_pointers_rejected_before_any_device_call(lib):
     p = ctypes.c_void_p(0)
     assert lib.dspark_draft_sample(p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_verify(p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
+    assert lib.dspark_draft_logits(p, p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, p, p, 0, p) == -1
+    assert lib.dspark_draft_pick(p, p, p, 4, 4, 1024, 0, 1, 0, 1, p, p, p, p, 0, p) == -1
     assert lib.dspark_prefix_schedule(p, p, p, 0.0, 4, 4, 0, 0.0, p, p, p, 0, p) == -1
     assert lib.dspark_read_status(p, p, None, None) == -1
     assert lib.dspark_clear_status(p, p) == -1

@@ -157,3 +157,34 @@ def test_masked_vocabulary_is_not_an_error(cuda_ok):
         emitted = out[out >= 0].long()
         assert not masked[emitted].any()
         assert not masked[rnd.x.cpu().long()].any()
+
+
+@pytest.mark.parametrize("greedy_frac", [0.0, 0.5])
+def test_split_draft_calls_match_draft_sample(cuda_ok, greedy_frac):
+    """dspark_draft_logits(k) then dspark_draft_pick(k) for k = 1..K gives
+    exactly dspark_draft_sample's outputs (tensor-core path at r = 256 and the
+    CUDA-core path at r = 272)."""
+    for r in (256, 272):
+        w = _small(B=130, V=4096, r=r, greedy_frac=greedy_frac)
+        inp = wl.generate(w)
+        dev = to_device(inp)
+        rnd = SpecRound(w.B, w.K, w.V, w.r)
+        rnd.run(dev, SEED, 3)
+        x = torch.full_like(rnd.x, -7)
+        d = torch.zeros_like(rnd.d)
+        q_lse = torch.zeros_like(rnd.q_lse)
+        q_tok = torch.zeros_like(rnd.q_tok)
+        ws = torch.zeros_like(rnd.ws)
+        for k in range(1, w.K + 1):
+            bn.draft_logits(dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], x,
+                            dev["temp"], k, d, ws)
+            bn.draft_pick(d, dev["last_tok"], dev["temp"], SEED, 3, k, x, q_lse, q_tok, ws)
+        torch.cuda.synchronize()
+        assert bn.read_status(ws) == (0, -1)
+        assert torch.equal(d, rnd.d) and torch.equal(x, rnd.x)
+        assert torch.equal(q_lse, rnd.q_lse) and torch.equal(q_tok, rnd.q_tok)
+        with pytest.raises(bn.DSparkError):
+            bn.draft_logits(dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], x,
+                            dev["temp"], w.K + 1, d, ws)
+        with pytest.raises(bn.DSparkError):
+            bn.draft_pick(d, dev["last_tok"], dev["temp"], SEED, 3, 0, x, q_lse, q_tok, ws)
