@@ -157,6 +157,10 @@ int dspark_draft_sample(const void* base, const void* U, const void* W, const fl
                             dtype, seed, round_id, x, d, q_lse, q_tok, ws, ws_bytes))
     return e;
   cudaStream_t s = (cudaStream_t)stream;
+  // one cooperative launch for the whole block when the tensor-core path
+  // applies and every M-tile gets its own CTAs; otherwise two launches per
+  // position (the same kernels, so the results are identical)
+  if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, s));
   for (int k = 1; k <= K; ++k) {
     cudaError_t e = launch_logits(a, k, sms, s);
     if (e == cudaSuccess) e = draft_sample_launch(a, k, s);

@@ -26,6 +26,7 @@ enum WaitSite : unsigned int {
   kWhereTcBaseEmpty = 13,
   kWhereTcAccFull = 14,
   kWhereTcAccEmpty = 15,
+  kWhereTcGrid = 16,
 };
 
 __device__ __forceinline__ void report_wait(Status* st, unsigned int site, int request) {
@@ -35,6 +36,9 @@ __device__ __forceinline__ void report_wait(Status* st, unsigned int site, int r
 }
 static_assert(sizeof(Status) == 256, "status block is 256 bytes");
 constexpr size_t kStatusBytes = 256;
+// Byte offset, inside the status block's padding, of the grid-barrier counter
+// of the one-launch draft round (zeroed by the launcher before each launch).
+constexpr size_t kGridBarrierOffset = 64;
 
 __device__ __forceinline__ void report(Status* st, unsigned int bits, int request) {
   atomicOr(&st->code, bits);

@@ -12,9 +12,11 @@
 //   draft_logits_*  d = round(base + scale * U[x_{k-1}] @ W) for a tile of
 //                   requests x 256 vocabulary entries, written to HBM, plus each
 //                   tile row's online-softmax partial (max, sum exp2) of d/temp
-//   draft_sample    per request: combine the chunk partials, locate the chunk
-//                   holding the inverse-CDF crossing, rescan that chunk (L2-hot)
+//   draft_sample    one warp per request: combine the chunk partials, locate
+//                   the chunk holding the inverse-CDF crossing, rescan that
+//                   chunk (L2-hot); see sample_warp.cuh
 #include "draft.cuh"
+#include "sample_warp.cuh"
 
 namespace dspark {
 
@@ -156,179 +158,12 @@ __global__ void __launch_bounds__(256) draft_logits_simt(DraftArgs a, int k) {
 }
 
 // ---------------------------------------------------------------------------
-// draft_sample: one block of 256 threads per request.
+// draft_sample: one warp per request, eight requests per block.
 // ---------------------------------------------------------------------------
 template <int DT>
 __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
-  using E = Elem<DT>;
-  using T = typename E::T;
-  __shared__ float wsum[8];
-  __shared__ float wmax[8];
-  __shared__ int wint[8];
-  __shared__ int s_owner;
-  __shared__ int s_chunk;
-  __shared__ float s_rem;
-  __shared__ int s_tok;
-  __shared__ int s_last;
-
-  const int b = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nch = a.nchunk;
-  const float2* P = a.partials + (long long)b * nch;
-  const float tau = a.temp[b];
-  const long long out_i = (long long)b * a.K + (k - 1);
-  Status* st = a.status;
-  if (tid == 0) {
-    if (tau != tau || tau < 0.f) report(st, DSPARK_STATUS_BAD_TEMP, b);
-    if (k == 1) {
-      const int lt = a.last_tok[b];
-      if (lt < 0 || lt >= a.V) report(st, DSPARK_STATUS_BAD_TOKEN, b);
-    }
-  }
-
-  if (!(tau > 0.f)) {
-    // greedy: argmax over the chunk partials
-    float mv = -INFINITY;
-    int mi = 0x7fffffff;
-    for (int c = tid; c < nch; c += 256) argmax_merge(mv, mi, P[c].x, __float_as_int(P[c].y));
-    bool bad = false;
-    for (int c = tid; c < nch; c += 256) bad |= (P[c].x != P[c].x);
-    warp_argmax(mv, mi);
-    const int anybad = __any_sync(0xffffffffu, bad);
-    if (lane == 0) {
-      wmax[warp] = mv;
-      wint[warp] = mi | (anybad ? 0x80000000 : 0);
-    }
-    __syncthreads();
-    if (tid == 0) {
-      float m = wmax[0];
-      int i = wint[0] & 0x7fffffff;
-      bool bb = wint[0] < 0;
-      for (int w = 1; w < 8; ++w) {
-        argmax_merge(m, i, wmax[w], wint[w] & 0x7fffffff);
-        bb |= wint[w] < 0;
-      }
-      if (bb || m == -INFINITY || i >= a.V) {
-        report(st, DSPARK_STATUS_BAD_ROW, b);
-        i = 0;
-      }
-      a.x[out_i] = i;
-      a.q_tok[out_i] = 1.f;
-      a.q_lse[out_i] = m;
-    }
-    return;
-  }
-
-  // contiguous range of chunks per thread (index order matters for the CDF)
-  const int per = (nch + 255) / 256;
-  const int c0 = min(tid * per, nch), c1 = min(c0 + per, nch);
-  float m = -INFINITY;
-  for (int c = c0; c < c1; ++c) m = fmaxf(m, P[c].x);
-  m = warp_max(m);
-  if (lane == 0) wmax[warp] = m;
-  __syncthreads();
-  float M = wmax[0];
-  for (int w = 1; w < 8; ++w) M = fmaxf(M, wmax[w]);
-
-  float s = 0.f;
-  for (int c = c0; c < c1; ++c) s += (P[c].x == -INFINITY) ? 0.f : P[c].y * ex2(P[c].x - M);
-  const float incl_w = warp_inclusive_scan(s);
-  if (lane == 31) wsum[warp] = incl_w;
-  __syncthreads();
-  float wpre = 0.f, Z = 0.f;
-  for (int w = 0; w < 8; ++w) {
-    if (w < warp) wpre += wsum[w];
-    Z += wsum[w];
-  }
-  const float excl = wpre + incl_w - s;
-
-  const bool badrow = !(Z > 0.f) || Z == INFINITY || M != M;
-  const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)k, kDraft);
-  const float thr = u * Z;
-  if (tid == 0) s_owner = 0x7fffffff;
-  __syncthreads();
-  if (!badrow && s > 0.f && thr < excl + s) atomicMin(&s_owner, tid);
-  __syncthreads();
-  const int owner = s_owner;
-  if (!badrow && owner != 0x7fffffff && tid == owner) {
-    // walk the owner's chunks in index order: first chunk whose mass exceeds
-    // what is left of u*Z
-    float rem = thr - excl;
-    int found = -1, lastpos = -1;
-    for (int c = c0; c < c1; ++c) {
-      const float vc = (P[c].x == -INFINITY) ? 0.f : P[c].y * ex2(P[c].x - M);
-      if (vc > 0.f) lastpos = c;
-      if (rem < vc) {
-        found = c;
-        break;
-      }
-      rem -= vc;
-    }
-    if (found < 0) {  // rounding: take the last positive element of the range
-      found = lastpos;
-      rem = INFINITY;
-    }
-    s_chunk = found;
-    s_rem = rem;
-  }
-  if (!badrow && owner == 0x7fffffff && tid == 0) {
-    // rounding: u*Z at or past the total; take the last positive element
-    int lastpos = -1;
-    for (int c = nch - 1; c >= 0; --c)
-      if (P[c].x != -INFINITY && P[c].y * ex2(P[c].x - M) > 0.f) {
-        lastpos = c;
-        break;
-      }
-    s_chunk = lastpos;
-    s_rem = INFINITY;
-  }
-  __syncthreads();
-  if (badrow) {
-    if (tid == 0) {
-      report(st, DSPARK_STATUS_BAD_ROW, b);
-      a.x[out_i] = 0;
-      a.q_tok[out_i] = 0.f;
-      a.q_lse[out_i] = NAN;
-    }
-    return;
-  }
-
-  // rescan the crossing chunk: one element per thread, block inclusive scan
-  const int ch = s_chunk;
-  const float rem = s_rem;
-  const float c = kLog2e / tau;
-  const int vi = ch * kChunk + tid;
-  const T* d = static_cast<const T*>(a.d);
-  float w = 0.f;
-  if (ch >= 0 && tid < kChunk && vi < a.V)
-    w = ex2(fmaf(E::load(d, ((long long)b * a.K + (k - 1)) * a.V + vi), c, -M));
-  const float iw = warp_inclusive_scan(w);
-  __syncthreads();
-  if (lane == 31) wsum[warp] = iw;
-  if (tid == 0) s_tok = 0x7fffffff;
-  __syncthreads();
-  float pre = 0.f;
-  for (int ww = 0; ww < warp; ++ww) pre += wsum[ww];
-  const float incl = pre + iw;
-  if (w > 0.f && rem < incl) atomicMin(&s_tok, tid);
-  __syncthreads();
-  int tok = s_tok;
-  if (tok == 0x7fffffff) {
-    // rounding fallback: last positive element of the chunk (a second
-    // variable: other threads may still be reading s_tok)
-    if (tid == 0) s_last = -1;
-    __syncthreads();
-    if (w > 0.f) atomicMax(&s_last, tid);
-    __syncthreads();
-    tok = s_last;
-  }
-  if (tid == (tok < 0 ? 0 : tok)) {
-    const int xi = (tok < 0) ? 0 : ch * kChunk + tok;
-    a.x[out_i] = xi;
-    a.q_tok[out_i] = w / Z;
-    a.q_lse[out_i] = M * 0.69314718055994530942f + logf(Z);
-    if (tok < 0) report(st, DSPARK_STATUS_BAD_ROW, b);
-  }
+  const int b = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (b < a.B) sample_row_warp<DT>(a, b, k);
 }
 
 // ---------------------------------------------------------------------------
@@ -354,9 +189,9 @@ cudaError_t draft_logits_simt_launch(const DraftArgs& a, int k, cudaStream_t s) 
 
 cudaError_t draft_sample_launch(const DraftArgs& a, int k, cudaStream_t s) {
   if (a.dtype == DSPARK_F32)
-    draft_sample<DSPARK_F32><<<a.B, 256, 0, s>>>(a, k);
+    draft_sample<DSPARK_F32><<<(a.B + 7) / 8, 256, 0, s>>>(a, k);
   else
-    draft_sample<DSPARK_BF16><<<a.B, 256, 0, s>>>(a, k);
+    draft_sample<DSPARK_BF16><<<(a.B + 7) / 8, 256, 0, s>>>(a, k);
   return cudaGetLastError();
 }
 

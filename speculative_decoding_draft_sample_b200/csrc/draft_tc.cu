@@ -32,6 +32,7 @@
 
 #include "draft.cuh"
 #include "draft_tc.cuh"
+#include "sample_warp.cuh"
 
 namespace dspark {
 
@@ -121,6 +122,11 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       "l"(map), "r"(su32(bar)), "r"(x), "r"(y), "r"(z), "l"(pol)
       : "memory");
 }
+// Pulls a W box into L2 ahead of its shared-memory load (no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
                                              int z, uint64_t pol) {
   asm volatile(
@@ -193,7 +199,26 @@ struct Params {
   float2* partials;        // [B, n_tiles]
   int nchunk;
   Status* status;
+  int k_last;              // positions p.k .. k_last in this launch
+  int fused;               // 1: sample every position in the kernel (grid barriers)
+  unsigned int* gbar;      // grid-barrier counter, zero at launch (fused only)
+  DraftArgs da;            // the draft call (sampling, next position's tokens)
 };
+
+// Grid-wide barrier of a cooperative launch, by one thread per CTA after a CTA
+// barrier: release (fence + arrival), then a bounded acquire spin until all
+// CTAs of barrier `n` (0-based) have arrived. False when the wait gave up.
+__device__ __forceinline__ bool grid_arrive_wait(unsigned int* ctr, unsigned int target) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+  const unsigned long long t0 = global_ns();
+  for (unsigned int it = 1;; ++it) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) break;
+    if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     draft_logits_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_base,
@@ -227,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nstride = p.ctas_per_m;
   const int n_my = (nt0 < p.n_tiles) ? (p.n_tiles - nt0 + nstride - 1) / nstride : 0;
   const int kblocks = (p.r + kWRows - 1) / kWRows;  // W stages per tile
+  const int npos = p.k_last - p.k + 1;  // draft positions in this launch
   const int ksteps = p.r / 16;           // MMAs per tile
 
   if (tid == 0) {
@@ -263,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     int last[kWStages];
     for (int q = 0; q < kWStages; ++q) last[q] = -1;
-    for (int i = 0; i < n_my; ++i) {
-      const int n0 = (nt0 + i * nstride) * kTileN;
+    for (int t = 0; t < n_my * npos; ++t) {  // W is the same at every position
+      const int n0 = (nt0 + (t % n_my) * nstride) * kTileN;
       bool stop = false;
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         const int s = it % kWStages;
@@ -280,6 +306,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int vb = 0; vb < 4; ++vb)
           tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + vb * 64, kb * kWRows, &w_full[s], pol_w);
         last[s] = it;
+        // the stage one ring-depth ahead goes to L2 now, so that its load
+        // (issued once a slot frees) is an L2 hit
+        {
+          const int it2 = it + kWStages;
+          const int t2 = it2 / kblocks;
+          if (t2 < n_my * npos) {
+            const int n2 = (nt0 + (t2 % n_my) * nstride) * kTileN;
+#pragma unroll
+            for (int vb = 0; vb < 4; ++vb) tma_prefetch_2d(&map_w, n2 + vb * 64, (it2 % kblocks) * kWRows);
+          }
+        }
       }
       if (stop) break;
     }
@@ -288,20 +325,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (last[q] >= 0) mbar_wait(&w_full[q], (last[q] / kWStages) & 1);
   } else if (warp == 2 && lane == 0) {
     // ---------------- base producer ----------------
-    // block j of tile i is block g = 4i + j of the ring (slot g % kBaseSlots)
+    // block j of tile t (counted over all positions) is block g = 4t + j of
+    // the ring (slot g % kBaseSlots)
     const uint64_t pol_base = policy_evict_first();
     int last[kBaseSlots];
     for (int q = 0; q < kBaseSlots; ++q) last[q] = -1;
-    for (int g = 0; g < 4 * n_my; ++g) {
+    for (int g = 0; g < 4 * n_my * npos; ++g) {
       const int s = g % kBaseSlots;
       if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[s], ((g / kBaseSlots) & 1) ^ 1)) {
         if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcBaseEmpty, m0);
         *(volatile int*)abort_flag = 1;
         break;
       }
-      const int n0 = (nt0 + (g >> 2) * nstride) * kTileN;
+      const int t = g >> 2;
+      const int n0 = (nt0 + (t % n_my) * nstride) * kTileN;
+      const int kpos = p.k + t / n_my;
       mbar_expect_tx(&b_full[s], kBlockBytes);
-      tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, p.k - 1, m0, &b_full[s], pol_base);
+      tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, kpos - 1, m0, &b_full[s], pol_base);
       last[s] = g;
     }
     if (*(volatile int*)abort_flag)
@@ -311,15 +351,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- MMA issuer ----------------
     // A is gathered by the epilogue warps meanwhile (the producers are already
     // streaming W and base); the whole warp waits for it at the named barrier
-    a_ready_sync();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (lane == 0) {
     int it = 0;
     int last_it = -1;  // last W stage whose MMAs were committed
     const uint32_t a_base = su32(sA);
+    for (int kp = 0; kp < npos; ++kp) {
+    a_ready_sync();  // A of this position is in shared memory
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (__shfl_sync(0xffffffffu, *(volatile int*)abort_flag, 0)) break;
+    if (lane == 0) {
     for (int i = 0; i < n_my; ++i) {
-      const int buf = i & 1;
-      if (*(volatile int*)abort_flag || !mbar_wait(&t_empty[buf], ((i >> 1) & 1) ^ 1)) {
+      const int ti = kp * n_my + i;  // tile counted over all positions
+      const int buf = ti & 1;
+      if (*(volatile int*)abort_flag || !mbar_wait(&t_empty[buf], ((ti >> 1) & 1) ^ 1)) {
         if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcAccEmpty, m0);
         *(volatile int*)abort_flag = 1;
         break;
@@ -367,10 +410,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               su32(&t_full[buf]))
           : "memory");
     }
-    // MMAs complete in order: once the last commit has landed, tensor memory is quiet
-    if (*(volatile int*)abort_flag && last_it >= 0)
-      mbar_wait(&w_empty[last_it % kWStages], (last_it / kWStages) & 1);
     }
+    __syncwarp();
+    }
+    // MMAs complete in order: once the last commit has landed, tensor memory is quiet
+    if (lane == 0 && *(volatile int*)abort_flag && last_it >= 0)
+      mbar_wait(&w_empty[last_it % kWStages], (last_it / kWStages) & 1);
   } else if (warp >= 4) {
     // ---------------- A gather, then the epilogue ----------------
     // A = U[prev_b, :] for the 128 rows of this M-tile, 128-byte swizzled,
@@ -379,12 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue warp e gathers rows 16e .. 16e + 15: lanes 0-15 read the rows'
     // tokens, then every lane loads one 16-byte chunk of each of the 16 rows
     // (all loads in flight at once; a row is one 512-byte coalesced read).
-    {
+    auto gather_a = [&](const int32_t* prev, int prev_stride) {
       const int ew = warp - 4;
       int tokv = 0;
       if (lane < 16) {
         const int b = m0 + ew * 16 + lane;
-        if (b < p.B) tokv = p.prev[(long long)b * p.prev_stride];
+        if (b < p.B) tokv = prev[(long long)b * prev_stride];
         if (tokv < 0 || tokv >= p.V) tokv = 0;  // reported by the sampler
       }
       const uint16_t* U = static_cast<const uint16_t*>(p.U);
@@ -403,8 +448,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(sA + kb * 16384 + m * 128 + ((c ^ (m & 7)) << 4)) = v[i];
       }
       fence_async_smem();
-      a_ready_arrive();
-    }
+    };
+    gather_a(p.prev, p.prev_stride);
+    a_ready_arrive();
     // ---------------- epilogue ----------------
     const int q = warp & 3;             // TMEM lane quadrant
     const int h = (warp - 4) >> 2;      // half: column blocks h and h + 2
@@ -419,11 +465,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool elected = (warp == 4 + 4 * h) && lane == 0;
     const uint64_t pol_d = policy_evict_first();
     bool miss = false;
+    bool aborted = false;
+    const bool leader = warp == 4 && lane == 0;
+    unsigned int nbar = 0;  // grid barriers passed
+    for (int kp = 0; kp < npos && !aborted; ++kp) {
+    const int kpos = p.k + kp;  // 1-based draft position
     for (int i = 0; i < n_my; ++i) {
+      const int ti = kp * n_my + i;  // tile counted over all positions
       const int nt = nt0 + i * nstride;
       const int n0 = nt * kTileN;
-      const int buf = i & 1;
-      if (!mbar_wait(&t_full[buf], (i >> 1) & 1)) {
+      const int buf = ti & 1;
+      if (!mbar_wait(&t_full[buf], (ti >> 1) & 1)) {
         miss = true;
         report_wait(p.status, kWhereTcAccFull, m0);
       }
@@ -436,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int jj = 0; jj < 2; ++jj) {
         const int j = h + 2 * jj;       // column block of the tile
-        const int g = 4 * i + j;        // block of the ring
+        const int g = 4 * ti + j;       // block of the ring
         const int slot = g % kBaseSlots;
         if (!mbar_wait(&b_full[slot], (g / kBaseSlots) & 1)) {
           miss = true;
@@ -526,27 +578,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         half_bar(h);
         if (elected) {
-          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, p.k - 1, m0, pol_d);
+          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, kpos - 1, m0, pol_d);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           if (jj == 1) {
             // the first block's store has read its slot: hand it back; the
             // second block's slot is handed back at the end of the tile
             asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-            mbar_arrive(&b_empty[(4 * i + h) % kBaseSlots]);
+            mbar_arrive(&b_empty[(4 * ti + h) % kBaseSlots]);
           }
         }
         __syncwarp();  // lane 0 may still be in the store above
       }
       if (elected) {
         asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        mbar_arrive(&b_empty[(4 * i + h + 2) % kBaseSlots]);
+        mbar_arrive(&b_empty[(4 * ti + h + 2) % kBaseSlots]);
       }
       __syncwarp();
       // this thread is done reading accumulator buffer `buf`
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&t_empty[buf]);
       // merge the two halves' statistics of this row
-      float2* xs = xstat + (i & 1) * 128;
+      float2* xs = xstat + (ti & 1) * 128;
       if (h == 1) {
         // greedy rows fold the NaN / +inf check into the max
         const bool bad_g = greedy && (chk != chk || chk == INFINITY);
@@ -556,6 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (epi_bar_any(miss)) {  // a wait gave up somewhere: every epilogue thread stops here
         *(volatile int*)abort_flag = 1;
+        aborted = true;
         break;
       }
       if (h == 0 && valid) {
@@ -577,6 +630,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         p.partials[(long long)b * p.nchunk + nt] = part;
       }
+    }
+    if (!aborted && p.fused) {
+      // this position's d is complete in global memory (the sampler reads it)
+      if (elected) {
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+      __syncwarp();
+      // every CTA's partials and d of this position -> sample -> every token
+      epi_bar_any(false);
+      bool fail = leader && !grid_arrive_wait(p.gbar, (++nbar) * gridDim.x);
+      if (fail) report_wait(p.status, kWhereTcGrid, m0);
+      aborted = epi_bar_any(fail);
+      if (!aborted) {
+        for (int rr = blockIdx.x + (warp - 4) * gridDim.x; rr < p.B; rr += 8 * gridDim.x)
+          sample_row_warp<DSPARK_BF16>(p.da, rr, kpos);
+        if (kp + 1 < npos) {
+          epi_bar_any(false);
+          fail = leader && !grid_arrive_wait(p.gbar, (++nbar) * gridDim.x);
+          if (fail) report_wait(p.status, kWhereTcGrid, m0);
+          aborted = epi_bar_any(fail);
+        }
+      }
+      if (aborted) *(volatile int*)abort_flag = 1;
+    }
+    if (kp + 1 < npos) {
+      // A of the next position from this position's tokens; on a failure the
+      // MMA warp still gets its arrival (it then sees the abort flag)
+      if (!aborted) gather_a(p.da.x + kpos - 1, p.da.K);
+      a_ready_arrive();
+    }
     }
     if (elected) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
@@ -625,40 +709,54 @@ bool draft_tc_supported(const DraftArgs& a) {
   return a.dtype == DSPARK_BF16 && a.r % 16 == 0 && a.r <= 256 && tc::encode_fn() != nullptr;
 }
 
-cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaStream_t s) {
+// Tensor maps and the fields of Params that every launch shares.
+static cudaError_t tc_setup(const DraftArgs& a, CUtensorMap* mw, CUtensorMap* mb, CUtensorMap* md,
+                            tc::Params* pp) {
   using namespace tc;
-  CUtensorMap mw, mb, md;
   {
     const cuuint64_t dims[2] = {(cuuint64_t)a.V, (cuuint64_t)a.r};
     const cuuint64_t strides[1] = {(cuuint64_t)a.V * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)kWRows};
-    if (!make_map(&mw, a.W, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_map(mw, a.W, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[3] = {(cuuint64_t)a.V, (cuuint64_t)a.K, (cuuint64_t)a.B};
     const cuuint64_t strides[2] = {(cuuint64_t)a.V * 2, (cuuint64_t)a.V * a.K * 2};
     const cuuint32_t box[3] = {64, 1, 128};
-    if (!make_map(&mb, a.base, 3, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!make_map(&md, a.d, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_map(mb, a.base, 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_map(md, a.d, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   cudaError_t e = cudaFuncSetAttribute(draft_logits_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
-  Params p;
+  Params& p = *pp;
   p.U = a.U;
-  p.prev = (k == 1) ? a.last_tok : a.x + (k - 2);
-  p.prev_stride = (k == 1) ? 1 : a.K;
   p.bias_scale = a.bias_scale;
   p.temp = a.temp;
   p.B = a.B;
   p.V = a.V;
   p.r = a.r;
-  p.k = k;
   p.m_tiles = (a.B + kTileM - 1) / kTileM;
   p.n_tiles = (a.V + kTileN - 1) / kTileN;
   p.partials = a.partials;
   p.nchunk = a.nchunk;
   p.status = a.status;
+  p.fused = 0;
+  p.gbar = nullptr;
+  p.da = a;
+  return cudaSuccess;
+}
+
+cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaStream_t s) {
+  using namespace tc;
+  CUtensorMap mw, mb, md;
+  Params p;
+  cudaError_t e = tc_setup(a, &mw, &mb, &md, &p);
+  if (e != cudaSuccess) return e;
+  p.prev = (k == 1) ? a.last_tok : a.x + (k - 2);
+  p.prev_stride = (k == 1) ? 1 : a.K;
+  p.k = k;
+  p.k_last = k;
   // launches of at most num_sms CTAs; each CTA keeps one M-tile (its A operand)
   for (int mf = 0; mf < p.m_tiles;) {
     const int m_here = min(p.m_tiles - mf, num_sms);
@@ -672,6 +770,44 @@ cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaS
     mf += m_here;
   }
   return cudaSuccess;
+}
+
+bool draft_round_tc_supported(const DraftArgs& a, int num_sms) {
+  return draft_tc_supported(a) && (a.B + tc::kTileM - 1) / tc::kTileM <= num_sms;
+}
+
+cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t s) {
+  using namespace tc;
+  CUtensorMap mw, mb, md;
+  Params p;
+  cudaError_t e = tc_setup(a, &mw, &mb, &md, &p);
+  if (e != cudaSuccess) return e;
+  if (p.m_tiles > num_sms) return cudaErrorInvalidValue;
+  p.prev = a.last_tok;
+  p.prev_stride = 1;
+  p.k = 1;
+  p.k_last = a.K;
+  p.fused = 1;
+  // the grid-barrier counter lives in the unused tail of the status block
+  p.gbar = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(a.status) + kGridBarrierOffset);
+  e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned int), s);
+  if (e != cudaSuccess) return e;
+  const int per_m = max(1, num_sms / p.m_tiles);
+  p.m_first = 0;
+  p.m_per_launch = p.m_tiles;
+  p.ctas_per_m = per_m;
+  // cooperative: every CTA is resident at once (one per SM), or the launch fails
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.m_tiles * per_m));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, draft_logits_tc, mw, mb, md, p);
 }
 
 }  // namespace dspark

@@ -10,5 +10,10 @@ namespace dspark {
 bool draft_tc_supported(const DraftArgs& a);
 // Draft logits and chunk partials of position k (1-based), persistent CTAs.
 cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaStream_t s);
+// True when all K positions fit one cooperative launch (M-tiles <= SMs).
+bool draft_round_tc_supported(const DraftArgs& a, int num_sms);
+// All K positions in one cooperative launch: logits, partials and the draw of
+// every position, with grid barriers between them.
+cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t s);
 
 }  // namespace dspark
