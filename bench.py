@@ -210,10 +210,11 @@ def main():
     dev = to_device(inp)
     rnd = SpecRound(w.B, w.K, w.V, w.r, torch.bfloat16)
     stream = torch.cuda.Stream()
+    side = torch.cuda.Stream()  # the prefix schedule runs here, beside the draft
     round_id = 0
 
     def step():
-        rnd.run(dev, wl.PHILOX_SEED, round_id, stream=stream)
+        rnd.run(dev, wl.PHILOX_SEED, round_id, stream=stream, side_stream=side)
 
     with torch.cuda.stream(stream):
         step()
@@ -276,25 +277,19 @@ def main():
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
             round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream), stream, 20)
 
-        # the dominant kernel alone: the draft-logit kernel of positions 1..K,
-        # one launch each (x already holds this round's tokens, so every
-        # launch sees the same inputs as in the round)
-        def logits_all():
-            for k in range(1, w.K + 1):
-                bn.draft_logits(dev["base"], dev["U"], dev["W"], dev["bias_scale"],
-                                dev["last_tok"], rnd.x, dev["temp"], k, rnd.d, rnd.ws, stream)
-        logits_all()
-        ms_logits = time_region(logits_all, stream, 10) / w.K
     # verify's algorithmic bytes: target rows 0..a_b of every request, plus the
     # draft row a_b of every request rejected before its cut
     rej = int((acc_np < cut).sum())
     verify_bytes = (int((acc_np + 1).sum()) + rej) * w.V * s_bytes
     verify_gbs = verify_bytes / (ms_verify * 1e-3) / 1e9
-    # draft-logit kernel, per launch: the base block in, d out, W once
-    logits_bytes = 2 * w.B * w.V * s_bytes + w.r * w.V * s_bytes
-    logits_gbs = logits_bytes / (ms_logits * 1e-3) / 1e9
-    draft_gbs = w.K * logits_bytes / (ms_draft * 1e-3) / 1e9
-    gemm_tflops = 2.0 * w.B * w.r * w.V / (ms_logits * 1e-3) / 1e12
+    # the draft kernel (one cooperative launch per round): per position the
+    # base block in, d out, W once, the chunk partials out and back in, the
+    # sampled chunk of d and the gathered U rows
+    nchunk = (w.V + 255) // 256
+    draft_bytes = w.K * (2 * w.B * w.V * s_bytes + w.r * w.V * s_bytes + 2 * w.B * nchunk * 8
+                         + w.B * 256 * s_bytes + w.B * w.r * s_bytes)
+    draft_gbs = draft_bytes / (ms_draft * 1e-3) / 1e9
+    gemm_tflops = 2.0 * w.B * w.r * w.V * w.K / (ms_draft * 1e-3) / 1e12
 
     # end to end through the public API from pinned host buffers
     host = to_device(inp, pin=True)
@@ -304,20 +299,21 @@ def main():
     d2h = out_h.numel() * 4 + n_h.numel() * 4
     with torch.cuda.stream(stream):
         for _ in range(2):
-            run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, stream=stream)
+            run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, stream=stream,
+                     side_stream=side)
         replicas.barrier()
         e2e_steps = max(3, args.steps // 5)
         ms_e2e = time_region(lambda: run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h,
-                                              stream=stream), stream, e2e_steps)
+                                              stream=stream, side_stream=side), stream, e2e_steps)
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
     traffic, traffic_src = profiled_traffic("draft_tc.cu", "draft_logits_tc_dspark5.txt")
-    roof = {"kernel": "draft_logits_tc (dspark_draft_logits, one draft position)", "bound": "hbm",
-            "achieved": logits_gbs, "peak": hbm, "unit": "GB/s", "frac": logits_gbs / hbm,
-            "traffic": traffic, "traffic_source": traffic_src,
+    roof = {"kernel": "draft_logits_tc (dspark_draft_sample: all K positions in one launch)",
+            "bound": "hbm", "achieved": draft_gbs, "peak": hbm, "unit": "GB/s",
+            "frac": draft_gbs / hbm, "traffic": traffic, "traffic_source": traffic_src,
             "peak_source": f"hbm_gbs of {peak_kind} peaks",
-            "bytes_per_launch": logits_bytes, "launch_ms": ms_logits,
-            "share_of_step": w.K * ms_logits / ms}
+            "bytes_per_launch": draft_bytes, "launch_ms": ms_draft,
+            "share_of_step": ms_draft / ms}
     line = {
         "metric": METRIC, "value": rounds_per_s, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -331,16 +327,15 @@ def main():
         "emitted_tok_per_s": emit_all * 1000.0 / ms,
         "accepted_per_round": accepted, "emitted_per_round": emitted,
         "mean_cut": float(cut.mean()), "mean_accepted": float(acc_np.mean()),
-        "stages_ms": {"draft": ms_draft, "draft_logits_per_launch": ms_logits,
-                      "schedule": ms_sched, "verify": ms_verify},
+        "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify},
         "verify": {"gbs": verify_gbs, "frac_of_hbm_peak": verify_gbs / hbm,
                    "bytes_per_launch": verify_bytes, "launch_ms": ms_verify},
-        "draft_stage": {"gbs": draft_gbs, "bias_gemm_tflops_per_launch": gemm_tflops,
+        "draft_stage": {"gbs": draft_gbs, "bias_gemm_tflops": gemm_tflops,
                         "bias_gemm_frac_of_bf16_peak": gemm_tflops / tflops},
         "roofline": roof,
         "e2e": {"value": world * 1000.0 / ms_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "gpu_launches": (2 * w.K + 2) * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

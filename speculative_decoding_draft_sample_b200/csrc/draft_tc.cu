@@ -39,6 +39,7 @@ namespace dspark {
 namespace tc {
 
 constexpr int kThreads = 384;      // 4 role warps + 8 epilogue warps
+constexpr int kFreeSms = 2;        // SMs the one-launch round leaves to other streams
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
 constexpr int kWRows = 32;          // Markov ranks per W stage
@@ -773,7 +774,7 @@ cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaS
 }
 
 bool draft_round_tc_supported(const DraftArgs& a, int num_sms) {
-  return draft_tc_supported(a) && (a.B + tc::kTileM - 1) / tc::kTileM <= num_sms;
+  return draft_tc_supported(a) && (a.B + tc::kTileM - 1) / tc::kTileM <= num_sms - tc::kFreeSms;
 }
 
 cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t s) {
@@ -792,7 +793,9 @@ cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t 
   p.gbar = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(a.status) + kGridBarrierOffset);
   e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned int), s);
   if (e != cudaSuccess) return e;
-  const int per_m = max(1, num_sms / p.m_tiles);
+  // kFreeSms SMs stay free for work on other streams (the prefix schedule,
+  // which needs none of the draft's outputs, runs there at the same time)
+  const int per_m = max(1, (num_sms - kFreeSms) / p.m_tiles);
   p.m_first = 0;
   p.m_per_launch = p.m_tiles;
   p.ctas_per_m = per_m;

@@ -39,16 +39,38 @@ class SpecRound:
         self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
 
     def run(self, inp: Dict[str, torch.Tensor], seed: int, round_id: int,
-            mode: int = bn.CUT_COST, threshold: float = 0.0, stream=None) -> None:
-        """Issues the round on ``stream`` (no host synchronisation)."""
+            mode: int = bn.CUT_COST, threshold: float = 0.0, stream=None,
+            side_stream=None) -> None:
+        """Issues the round on ``stream`` (no host synchronisation).
+
+        The prefix schedule needs only the confidence logits, so with a
+        ``side_stream`` it runs there, concurrently with the draft (the
+        one-launch draft kernel leaves SMs free for it); verification waits
+        for both. The two calls share the workspace: they only meet in its
+        status block, which both update atomically.
+        """
+        main = stream if stream is not None else torch.cuda.current_stream()
+
+        def schedule(s):
+            bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
+                               float(inp["fixed_cost"]), mode, threshold, self.cut, self.survival,
+                               self.ws, s)
+
+        if side_stream is not None:
+            fork, join = torch.cuda.Event(), torch.cuda.Event()
+            fork.record(main)
+            side_stream.wait_event(fork)
+            schedule(side_stream)
+            join.record(side_stream)
         bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
                         inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
-                        self.ws, stream)
-        bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
-                           float(inp["fixed_cost"]), mode, threshold, self.cut, self.survival,
-                           self.ws, stream)
+                        self.ws, main)
+        if side_stream is None:
+            schedule(main)
+        else:
+            main.wait_event(join)
         bn.verify(inp["target"], self.d, self.x, self.q_tok, self.cut, inp["temp"], seed,
-                  round_id, self.accepted, self.out, self.n_emit, self.ws, stream)
+                  round_id, self.accepted, self.out, self.n_emit, self.ws, main)
 
     def status(self, stream=None):
         return bn.read_status(self.ws, stream)
@@ -76,10 +98,10 @@ def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -
 
 def run_host(rnd: SpecRound, host: Dict[str, object], dev: Dict[str, object], seed: int,
              round_id: int, out_host: torch.Tensor, n_emit_host: torch.Tensor,
-             mode: int = bn.CUT_COST, stream=None) -> None:
+             mode: int = bn.CUT_COST, stream=None, side_stream=None) -> None:
     """End to end from pinned host buffers: H2D copies, the round, D2H of the tokens."""
     for k in DEVICE_KEYS:
         dev[k].copy_(host[k], non_blocking=True)
-    rnd.run(dev, seed, round_id, mode, stream=stream)
+    rnd.run(dev, seed, round_id, mode, stream=stream, side_stream=side_stream)
     out_host.copy_(rnd.out, non_blocking=True)
     n_emit_host.copy_(rnd.n_emit, non_blocking=True)

@@ -188,3 +188,21 @@ def test_split_draft_calls_match_draft_sample(cuda_ok, greedy_frac):
                             dev["temp"], w.K + 1, d, ws)
         with pytest.raises(bn.DSparkError):
             bn.draft_pick(d, dev["last_tok"], dev["temp"], SEED, 3, 0, x, q_lse, q_tok, ws)
+
+
+def test_schedule_on_side_stream_matches_one_stream(cuda_ok):
+    """The prefix schedule issued on a side stream, concurrently with the draft
+    (sharing the workspace), gives the same round as one stream."""
+    w = _small(B=200, V=8192)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    a = SpecRound(w.B, w.K, w.V, w.r)
+    a.run(dev, SEED, 5)
+    b = SpecRound(w.B, w.K, w.V, w.r)
+    main, side = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(main):
+        b.run(dev, SEED, 5, stream=main, side_stream=side)
+    torch.cuda.synchronize()
+    assert a.status() == (0, -1) and b.status() == (0, -1)
+    for name in ("x", "d", "q_tok", "cut", "survival", "accepted", "out", "n_emit"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
