@@ -103,6 +103,22 @@ __device__ __forceinline__ uint32_t philox_word0(uint32_t c0, uint32_t c1, uint3
   return c0;
 }
 
+// Grid-wide barrier of a cooperative launch, by one thread per CTA after a
+// CTA barrier: a release arrival on a counter that is zero at launch, then a
+// bounded acquire spin until every CTA of barrier number n (1-based; target
+// n * gridDim.x) has arrived. False when the wait gave up.
+__device__ __forceinline__ bool grid_arrive_wait(unsigned int* ctr, unsigned int target) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+  const unsigned long long t0 = global_ns();
+  for (unsigned int it = 1;; ++it) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) break;
+    if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
 enum Purpose : uint32_t { kDraft = 0, kAccept = 1, kResidual = 2, kBonus = 3 };
 
 // The round's 24-bit uniform for (request, position, purpose); exact in fp32.

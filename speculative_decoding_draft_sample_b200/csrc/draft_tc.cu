@@ -206,20 +206,7 @@ struct Params {
   DraftArgs da;            // the draft call (sampling, next position's tokens)
 };
 
-// Grid-wide barrier of a cooperative launch, by one thread per CTA after a CTA
-// barrier: release (fence + arrival), then a bounded acquire spin until all
-// CTAs of barrier `n` (0-based) have arrived. False when the wait gave up.
-__device__ __forceinline__ bool grid_arrive_wait(unsigned int* ctr, unsigned int target) {
-  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-  const unsigned long long t0 = global_ns();
-  for (unsigned int it = 1;; ++it) {
-    unsigned int v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    if (v >= target) break;
-    if ((it & 255u) == 0 && global_ns() - t0 > kWaitLimitNs) return false;
-  }
-  return true;
-}
+
 
 __global__ void __launch_bounds__(kThreads, 1)
     draft_logits_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_base,
