@@ -8,13 +8,15 @@
 // online-softmax partial (max, sum exp2) of d * log2(e) / temperature, or
 // (max, argmax) for greedy requests.
 //
-// GEMM shape: M = requests (128 per tile), N = vocabulary (256 per tile),
-// K = Markov rank (<= 256). A = the gathered U rows (K-major, built in shared
-// memory once per CTA), B = W (vocabulary-major; tiles arrive by TMA with
-// 128-byte swizzle), D = fp32 in tensor memory (two 256-column buffers).
+// GEMM shape: M = requests (128 per tile), N = vocabulary (256 per tile, as
+// two MMA halves of 128), K = Markov rank (<= 256). A = the gathered U rows
+// (K-major, built in shared memory once per position), B = W (vocabulary-
+// major; stages arrive by TMA with 128-byte swizzle), D = fp32 in tensor
+// memory (two 256-column buffers).
 //
 // Persistent CTAs, one per SM, warp-specialised:
-//   warp 0     TMA producer of W tiles (ring of four 16 KB stages of 32 ranks)
+//   warp 0     TMA producer of W tiles (ring of four 16 KB stages of 64 ranks x
+//              128 vocabulary entries: one vocabulary half of a tile per four stages)
 //   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer (it
 //              waits at a named barrier for A, which the epilogue warps gather
 //              while the producers already stream W and base)
@@ -42,10 +44,11 @@ constexpr int kThreads = 384;      // 4 role warps + 8 epilogue warps
 constexpr int kFreeSms = 2;        // SMs the one-launch round leaves to other streams
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
-constexpr int kWRows = 32;          // Markov ranks per W stage
-constexpr int kWStages = 4;         // W ring depth (stages of 32 ranks x 256 vocab)
-constexpr int kWStageBytes = kWRows * 256 * 2;
-constexpr int kWBoxBytes = kWRows * 64 * 2;  // one [32 x 64] TMA box
+constexpr int kWRows = 64;          // Markov ranks per W stage
+constexpr int kWCols = 128;         // vocabulary columns per W stage (one MMA half)
+constexpr int kWStages = 4;         // W ring depth (stages of 64 ranks x 128 vocab)
+constexpr int kWStageBytes = kWRows * kWCols * 2;
+constexpr int kWBoxBytes = kWRows * 64 * 2;  // one [64 ranks x 64 vocab] TMA box
 constexpr int kBaseSlots = 6;       // base/d ring of [128 x 64] blocks: 1.5 tiles
 constexpr int kBlockBytes = 128 * 64 * 2;
 constexpr int kABytes = 128 * 256 * 2;  // gathered U rows, 4 k-blocks of [128 x 64]
@@ -55,15 +58,16 @@ constexpr int kOffA = 0;
 constexpr int kOffW = kOffA + kABytes;
 constexpr int kOffBase = kOffW + kWStages * kWStageBytes;
 constexpr int kOffBar = kOffBase + kBaseSlots * kBlockBytes;
-constexpr int kNumBars = 2 * kWStages + 2 * kBaseSlots + 4;
+constexpr int kNumBars = 2 * kWStages + 2 * kBaseSlots + 6;
 constexpr int kOffX = kOffBar + kNumBars * 8 + 16;              // [2][128] float2 row stats
 constexpr int kSmemBytes = kOffX + 2 * 128 * 8;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
 
 // instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 MN-major,
-// M = 128, N = 256
+// M = 128, N = 128 (a tile's accumulator is two such halves, committed apart,
+// so that the epilogue starts on the first half while W of the second arrives)
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) |
-                            ((uint32_t)(kTileN >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
+                            ((uint32_t)(kWCols >> 3) << 17) | ((uint32_t)(kTileM >> 4) << 24);
 
 __device__ __forceinline__ uint32_t su32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -226,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* w_empty = bars + kWStages;
   uint64_t* b_full = bars + 2 * kWStages;
   uint64_t* b_empty = b_full + kBaseSlots;
-  uint64_t* t_full = b_empty + kBaseSlots;   // [2]
-  uint64_t* t_empty = t_full + 2;            // [2]
+  uint64_t* t_full = b_empty + kBaseSlots;   // [2 buffers][2 halves]
+  uint64_t* t_empty = t_full + 4;            // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float2* xstat = reinterpret_cast<float2*>(smem + kOffX);
@@ -239,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nt0 = blockIdx.x / p.m_per_launch;
   const int nstride = p.ctas_per_m;
   const int n_my = (nt0 < p.n_tiles) ? (p.n_tiles - nt0 + nstride - 1) / nstride : 0;
-  const int kblocks = (p.r + kWRows - 1) / kWRows;  // W stages per tile
+  const int kbh = (p.r + kWRows - 1) / kWRows;  // W stages per MMA half
+  const int kblocks = 2 * kbh;                   // W stages per tile
   const int npos = p.k_last - p.k + 1;  // draft positions in this launch
   const int ksteps = p.r / 16;           // MMAs per tile
 
@@ -252,10 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&b_full[i], 1);
       mbar_init(&b_empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&t_full[i], 1);
-      mbar_init(&t_empty[i], 256);
-    }
+    for (int i = 0; i < 4; ++i) mbar_init(&t_full[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&t_empty[i], 256);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -290,9 +293,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_expect_tx(&w_full[s], kWStageBytes);
         unsigned char* dst = sW + s * kWStageBytes;
+        // stage kb: ranks (kb % kbh) * 64 .. + 63 of vocabulary half kb / kbh
 #pragma unroll
-        for (int vb = 0; vb < 4; ++vb)
-          tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + vb * 64, kb * kWRows, &w_full[s], pol_w);
+        for (int vb = 0; vb < 2; ++vb)
+          tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + (kb / kbh) * kWCols + vb * 64,
+                      (kb % kbh) * kWRows, &w_full[s], pol_w);
         last[s] = it;
         // the stage one ring-depth ahead goes to L2 now, so that its load
         // (issued once a slot frees) is an L2 hit
@@ -301,8 +306,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t2 = it2 / kblocks;
           if (t2 < n_my * npos) {
             const int n2 = (nt0 + (t2 % n_my) * nstride) * kTileN;
+            const int kb2 = it2 % kblocks;
 #pragma unroll
-            for (int vb = 0; vb < 4; ++vb) tma_prefetch_2d(&map_w, n2 + vb * 64, (it2 % kblocks) * kWRows);
+            for (int vb = 0; vb < 2; ++vb)
+              tma_prefetch_2d(&map_w, n2 + (kb2 / kbh) * kWCols + vb * 64, (kb2 % kbh) * kWRows);
           }
         }
       }
@@ -356,9 +363,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t d_tmem = tmem + buf * kTileN;
       bool ok = true;
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int hh = kb / kbh, rb = kb % kbh;  // vocabulary half, rank block
+        const uint32_t d_tmem = tmem + buf * kTileN + hh * kWCols;
         const int s = it % kWStages;
         if (!mbar_wait(&w_full[s], (it / kWStages) & 1)) {
           report_wait(p.status, kWhereTcWFull, m0);
@@ -369,11 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t w_base = su32(sW + s * kWStageBytes);
 #pragma unroll
         for (int kk = 0; kk < kWRows / 16; ++kk) {
-          const int step = kb * (kWRows / 16) + kk;  // 16 ranks per MMA
+          const int step = rb * (kWRows / 16) + kk;  // 16 ranks per MMA
           if (step < ksteps) {
-            // A: 64-rank sub-tile step / 4, 32-byte step inside its 128-byte swizzle row
-            const uint64_t ad = sdesc(a_base + (step >> 2) * 16384 + (step & 3) * 32, 16, 1024);
-            // B: 16 k-rows (2 groups of 8) per step; 64-vocab boxes kWBoxBytes apart
+            // A: 64-rank sub-tile rb, 32-byte step kk inside its 128-byte swizzle row
+            const uint64_t ad = sdesc(a_base + rb * 16384 + kk * 32, 16, 1024);
+            // B: 16 k-rows (2 groups of 8) per step; the two 64-vocab boxes kWBoxBytes apart
             const uint64_t bd = sdesc(w_base + kk * 2048, kWBoxBytes, 1024);
             const uint32_t acc = (step > 0) ? 1u : 0u;
             asm volatile(
@@ -388,15 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 su32(&w_empty[s]))
             : "memory");
         last_it = it;
+        if (rb == kbh - 1)  // this half of the accumulator is complete
+          asm volatile(
+              "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                  su32(&t_full[2 * buf + hh]))
+              : "memory");
       }
       if (!ok) {
         *(volatile int*)abort_flag = 1;
         break;
       }
-      asm volatile(
-          "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-              su32(&t_full[buf]))
-          : "memory");
     }
     }
     __syncwarp();
@@ -463,12 +472,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int nt = nt0 + i * nstride;
       const int n0 = nt * kTileN;
       const int buf = ti & 1;
-      if (!mbar_wait(&t_full[buf], (ti >> 1) & 1)) {
-        miss = true;
-        report_wait(p.status, kWhereTcAccFull, m0);
-      }
-      __syncwarp();
-      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       // sampled rows: running max of z = d * cs and sum of 2^(z - max)
       // greedy rows: running (max d, argmax), NaN-propagating check value
       float run_m = -INFINITY, run_s = 0.f, chk = -INFINITY;
@@ -482,7 +485,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           miss = true;
           report_wait(p.status, kWhereTcBaseFull, m0);
         }
+        // column block j lies in MMA half jj: wait for that half's commit
+        if (!mbar_wait(&t_full[2 * buf + jj], (ti >> 1) & 1)) {
+          miss = true;
+          report_wait(p.status, kWhereTcAccFull, m0);
+        }
         __syncwarp();  // tcgen05.ld is warp-aligned: every lane, together
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         float acc[64];
         const uint32_t col = tmem + lane_base + buf * kTileN + j * 64;
         tmem_ld32(col, acc);
