@@ -467,6 +467,49 @@ __device__ __forceinline__ float2 combine_ranks(const Exch* got, int C) {
   return make_float2(M, Z);
 }
 
+// Cluster q verifies the request of rank q in the order (cut descending,
+// index ascending): the longest chains of rows start in the first wave of
+// clusters and the requests that verify a single row take the slots that free
+// up last. Every CTA of the cluster computes the same answer: a histogram of
+// the (clamped) cuts, the cut value whose range holds q, then the position of
+// the request among those with that cut, in index order.
+__device__ int request_of(const VerifyArgs& a, int q, int* cnt, int* s_req) {
+  if (!a.cut) return q;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int K = a.K;
+  for (int v = tid; v <= K; v += kVThreads) cnt[v] = 0;
+  __syncthreads();
+  for (int i = tid; i < a.B; i += kVThreads) {
+    const int L = min(max(a.cut[i], 0), K);
+    atomicAdd(&cnt[L], 1);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // the cut value v whose rank range [base, base + cnt[v]) holds q
+    int base = 0, v = K;
+    for (; v > 0 && q >= base + cnt[v]; --v) base += cnt[v];
+    // the (q - base)-th request with cut v, in index order
+    int want = q - base, found = -1;
+    for (int i0 = 0; i0 < a.B && found < 0; i0 += 32) {
+      const int i = i0 + lane;
+      const bool hit = i < a.B && min(max(a.cut[i], 0), K) == v;
+      const unsigned m = __ballot_sync(0xffffffffu, hit);
+      const int n = __popc(m);
+      if (want < n) {
+        unsigned mm = m;
+        for (int k = 0; k < want; ++k) mm &= mm - 1;
+        found = i0 + __ffs(mm) - 1;
+      } else {
+        want -= n;
+      }
+    }
+    if (lane == 0) *s_req = found < 0 ? q : found;
+  }
+  (void)warp;
+  __syncthreads();
+  return *s_req;
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(VerifyArgs a) {
   using E = Elem<DT>;
@@ -481,6 +524,8 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   __shared__ float red[32];
   __shared__ int sint[4];
   __shared__ int dead;
+  __shared__ int cnt_by_cut[65];
+  __shared__ int s_req;
 
   VerifyCta<DT> c;
   c.C = cluster_size();
@@ -501,7 +546,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   c.parity = 0;
   c.issued = 0;
   c.consumed = 0;
-  const int b = blockIdx.x / c.C;
+  const int b = request_of(a, blockIdx.x / c.C, cnt_by_cut, &s_req);
   c.request = b;
   c.lo = c.rank * a.slice;
   c.n = max(0, min(a.slice, a.V - c.lo));
