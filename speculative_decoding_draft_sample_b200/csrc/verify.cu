@@ -11,6 +11,8 @@
 //
 // Design (B200): one thread-block cluster of C small CTAs (128 threads) per
 // request; CTA `rank` owns vocabulary slice [rank*slice, rank*slice + slice).
+// Clusters take requests in descending order of their cut, so that the
+// longest chains of rows start in the first wave of resident clusters.
 // A request's target rows are walked in order and the walk stops at the first
 // rejection, so HBM sees only rows 0..a and one draft row. Each slice streams
 // through a ring of 8 KB shared-memory slots filled by bulk asynchronous copies
