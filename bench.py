@@ -189,6 +189,34 @@ def reference_arm(args, w: wl.Workload):
     print(json.dumps(line), flush=True)
 
 
+def load_sweep():
+    """NEXT-3 of the scheduler: how the early-stopping cut trims the verified
+    block as the batch grows, against the DSpark-5 cost table (a step in the
+    per-token cost at 512 verified tokens). Prefix schedule only; one JSON line
+    per batch size."""
+    torch.cuda.set_device(0)
+    stream = torch.cuda.Stream()
+    for B in (32, 64, 128, 256, 512, 1024):
+        w = wl.scaled(wl.DSPARK5, name=f"load_b{B}", B=B)
+        small = wl.small_inputs(w)
+        dev = {k: torch.as_tensor(small[k]).cuda() for k in ("conf_logit", "pos_temp", "step_cost")}
+        cut = torch.empty(B, dtype=torch.int32, device="cuda")
+        surv = torch.empty((B, w.K), dtype=torch.float32, device="cuda")
+        ws = torch.zeros(bn.workspace_bytes(bn.OP_SCHEDULE, B, w.K, 8, 1, bn.F32), dtype=torch.uint8,
+                         device="cuda")
+        def call():
+            bn.prefix_schedule(dev["conf_logit"], dev["pos_temp"], dev["step_cost"],
+                               small["fixed_cost"], bn.CUT_COST, 0.0, cut, surv, ws, stream)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                call()
+            ms = time_region(call, stream, 20)
+        c = cut.cpu().numpy()
+        print(json.dumps({"B": B, "K": w.K, "mean_cut": float(c.mean()),
+                          "verified_tokens": int(c.sum() + B), "schedule_us": ms * 1e3,
+                          "cut_hist": np.bincount(c, minlength=w.K + 1).tolist()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -196,8 +224,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=wl.DSPARK5.name, choices=sorted(wl.ALL),
+                    help="measure another configuration (the default is the headline one)")
+    ap.add_argument("--load-sweep", action="store_true",
+                    help="prefix schedule only: mean cut and time as the batch grows")
     args = ap.parse_args()
-    w = wl.DSPARK5
+    if args.load_sweep:
+        load_sweep()
+        return
+    w = wl.ALL[args.workload]
     if args.impl == "reference":
         reference_arm(args, w)
         return
@@ -208,7 +243,8 @@ def main():
     # each rank: its own batch (weak scaling), no collective on the data path
     inp = wl.generate(replicas.rank_workload(w, rank))
     dev = to_device(inp)
-    rnd = SpecRound(w.B, w.K, w.V, w.r, torch.bfloat16)
+    tdt = torch.float32 if w.dtype == wl.F32 else torch.bfloat16
+    rnd = SpecRound(w.B, w.K, w.V, w.r, tdt)
     stream = torch.cuda.Stream()
     side = torch.cuda.Stream()  # the prefix schedule runs here, beside the draft
     round_id = 0
@@ -264,7 +300,7 @@ def main():
     rounds_per_s = world * 1000.0 / ms
 
     # per-stage times (same stream, CUDA events), each stage alone
-    s_bytes = 2
+    s_bytes = w.nbytes_per_logit
     with torch.cuda.stream(stream):
         ms_draft = time_region(lambda: bn.draft_sample(
             dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], dev["temp"],
@@ -307,7 +343,10 @@ def main():
                                               stream=stream, side_stream=side), stream, e2e_steps)
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
+    in_bytes = (w.B * (w.K + 1) * w.V + w.B * w.K * w.V + 2 * w.V * w.r) * s_bytes
     traffic, traffic_src = profiled_traffic("draft_tc.cu", "draft_logits_tc_dspark5.txt")
+    if w.name != wl.DSPARK5.name:
+        traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload only"
     roof = {"kernel": "draft_logits_tc (dspark_draft_sample: all K positions in one launch)",
             "bound": "hbm", "achieved": draft_gbs, "peak": hbm, "unit": "GB/s",
             "frac": draft_gbs / hbm, "traffic": traffic, "traffic_source": traffic_src,
@@ -317,11 +356,14 @@ def main():
     line = {
         "metric": METRIC, "value": rounds_per_s, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == wl.F32 else "bf16",
         "data": "synthetic (seeded Zipf+noise logits, random Markov factors)",
         "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
                    "global_batch": w.B * world, "parallelism": f"replicas{world}",
-                   "l2": "inputs (728 MB) larger than L2 (126 MB); not flushed",
+                   "l2": (f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2 (126 MB); not flushed"
+                          if in_bytes > L2_BYTES else
+                          f"inputs ({in_bytes / 1e6:.0f} MB) fit in L2 (126 MB); not flushed"),
                    "timing": "CUDA graph of the round, CUDA events, max over ranks"},
         "accepted_tok_per_s": acc_all * 1000.0 / ms,
         "emitted_tok_per_s": emit_all * 1000.0 / ms,
@@ -338,7 +380,7 @@ def main():
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name:
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), 128, 0).items()
                                 if k in ("value", "unit", "cores", "kind", "sample")}
     del graph  # released before the process group goes away
