@@ -231,3 +231,24 @@ def generate(w: Workload, requests: Optional[List[int]] = None) -> Dict[str, obj
             fill(ib)
     out.update(target=target, base=base, requests=reqs)
     return out
+
+
+# ---------------------------------------------------------------------------
+# Calibration data for Sequential Temperature Scaling: a synthetic confidence
+# head that is over-confident by a factor gamma_k at position k. Latent
+# per-position survival probabilities pi = sigmoid(mu_k + 1.2 eps), labels
+# survived[n, k] = survived[n, k-1] and Bernoulli(pi[n, k]), confidence
+# logits z = gamma_k * logit(pi) (so that z / gamma_k is calibrated).
+# ---------------------------------------------------------------------------
+CALIB_GAMMAS = (1.6, 1.9, 2.2, 2.5, 2.8)
+
+
+def calib_inputs(N: int, K: int = 5, gammas=CALIB_GAMMAS, seed: int = 3):
+    rng = np.random.default_rng([seed, 29])
+    mu = 1.0 - 0.25 * np.arange(K)
+    logit_pi = mu[None, :] + 1.2 * rng.standard_normal((N, K))
+    pi = 1.0 / (1.0 + np.exp(-logit_pi))
+    draw = rng.random((N, K)) < pi
+    survived = np.cumprod(draw, axis=1).astype(np.uint8)
+    z = (np.asarray(gammas[:K], np.float64)[None, :] * logit_pi).astype(np.float32)
+    return z, survived
