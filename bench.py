@@ -217,6 +217,28 @@ def load_sweep():
                           "cut_hist": np.bincount(c, minlength=w.K + 1).tolist()}), flush=True)
 
 
+def calib_bench(N: int):
+    """Sequential Temperature Scaling (dspark_sts_fit) on N synthetic samples of
+    an over-confident head: CUDA-event time and the ECE before / after."""
+    torch.cuda.set_device(0)
+    K = 5
+    z, y = wl.calib_inputs(N, K=K)
+    zt, yt = torch.from_numpy(z).cuda(), torch.from_numpy(y).cuda()
+    T = torch.zeros(K, device="cuda")
+    idx = torch.zeros(K, dtype=torch.int32, device="cuda")
+    eb, ea = torch.zeros(K, device="cuda"), torch.zeros(K, device="cuda")
+    ws = torch.zeros(bn.workspace_bytes(bn.OP_CALIB, N, K, 0, 0, 0), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            bn.sts_fit(zt, yt, T, idx, eb, ea, ws, stream)
+        ms = time_region(lambda: bn.sts_fit(zt, yt, T, idx, eb, ea, ws, stream), stream, 10)
+    print(json.dumps({"N": N, "K": K, "ms": ms, "samples_x_grid_per_s": 256 * N * K / (ms * 1e-3),
+                      "T": T.cpu().tolist(), "ece_before": eb.cpu().tolist(),
+                      "ece_after": ea.cpu().tolist(), "launches": 2 * K + 4,
+                      "loss_evaluations": 256 * N * K}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -228,9 +250,14 @@ def main():
                     help="measure another configuration (the default is the headline one)")
     ap.add_argument("--load-sweep", action="store_true",
                     help="prefix schedule only: mean cut and time as the batch grows")
+    ap.add_argument("--calib", type=int, default=0, metavar="N",
+                    help="Sequential Temperature Scaling of N synthetic samples (K = 5): time and ECE")
     args = ap.parse_args()
     if args.load_sweep:
         load_sweep()
+        return
+    if args.calib:
+        calib_bench(args.calib)
         return
     w = wl.ALL[args.workload]
     if args.impl == "reference":

@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdspark.so")
 
 F32, BF16 = 0, 1
-OP_DRAFT, OP_SCHEDULE, OP_VERIFY = 0, 1, 2
+OP_DRAFT, OP_SCHEDULE, OP_VERIFY, OP_CALIB = 0, 1, 2, 3
 CUT_COST, CUT_THRESHOLD, CUT_NONE = 0, 1, 2
 STATUS_BAD_TOKEN, STATUS_BAD_ROW, STATUS_BAD_CUT, STATUS_BAD_TEMP, STATUS_TIMEOUT = 1, 2, 4, 8, 16
 STATUS_INTERNAL = 32
@@ -44,6 +44,7 @@ SIGNATURES = {
                                _p]),
     "dspark_draft_sample_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
                                         _p, _p, _p, _p, _p, _p]),
+    "dspark_sts_fit": (_i, [_p, _p, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
     "dspark_read_status": (_i, [_p, _p, ctypes.POINTER(ctypes.c_uint32),
                                 ctypes.POINTER(ctypes.c_int32)]),
     "dspark_clear_status": (_i, [_p, _p]),
@@ -196,6 +197,17 @@ def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, o
         _ptr(n_emit, "n_emit", torch.int32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
         _stream(stream))
     _check(rc, "dspark_verify")
+
+
+def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, stream=None) -> None:
+    """dspark_sts_fit: conf_logit [N,K] f32, survived [N,K] u8 -> T [K], index [K], ECE [K] x 2."""
+    N, K = conf_logit.shape
+    rc = lib().dspark_sts_fit(
+        _ptr(conf_logit, "conf_logit", torch.float32), _ptr(survived, "survived", torch.uint8), N, K,
+        _ptr(T_out, "T_out", torch.float32), _ptr(index_out, "index_out", torch.int32),
+        _ptr(ece_before, "ece_before", torch.float32), _ptr(ece_after, "ece_after", torch.float32),
+        _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    _check(rc, "dspark_sts_fit")
 
 
 def read_status(ws, stream=None) -> Tuple[int, int]:

@@ -3,6 +3,7 @@
 #include <climits>
 #include <cstring>
 
+#include "calib.cuh"
 #include "common.cuh"
 #include "draft.cuh"
 #include "draft_tc.cuh"
@@ -70,6 +71,9 @@ size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype) {
     case DSPARK_OP_SCHEDULE:
       if (B < 1 || K < 1 || K > 64) return 0;
       return kStatusBytes;
+    case DSPARK_OP_CALIB:
+      if (B < 1 || K < 1 || K > 64) return 0;
+      return calib_workspace_bytes(B, K);
     case DSPARK_OP_VERIFY:
       if (!shape_ok(B, K, V, dtype)) return 0;
       return kStatusBytes;
@@ -253,6 +257,25 @@ int dspark_verify(const void* target, const void* d, const int32_t* x, const flo
   a.status = static_cast<Status*>(ws);
   const int C = verify_cluster_size(B, V, dtype, sms);
   return cuda_status(verify_launch(a, C, (cudaStream_t)stream));
+}
+
+int dspark_sts_fit(const float* conf_logit, const uint8_t* survived, int N, int K, float* T_out,
+                   int32_t* index_out, float* ece_before, float* ece_after, void* ws,
+                   size_t ws_bytes, dspark_stream_t stream) {
+  if (!conf_logit || !survived || !T_out || !ws) return DSPARK_ERR_INVALID_ARG;
+  if (N < 1 || K < 1 || K > 64) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_CALIB, N, K, 8, 1, DSPARK_F32))
+    return DSPARK_ERR_WORKSPACE;
+  if (int e = device_check(nullptr)) return e;
+  CalibArgs a;
+  a.z = conf_logit;
+  a.y = survived;
+  a.N = N;
+  a.K = K;
+  a.T = T_out;
+  a.index = index_out;
+  return cuda_status(calib_launch(a, ws, ece_before, ece_after, (cudaStream_t)stream));
 }
 
 }  // extern "C"

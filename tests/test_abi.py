@@ -46,6 +46,9 @@ def test_workspace_sizes(lib):
     assert bn.workspace_bytes(bn.OP_DRAFT, 4, 4, 1001, 16, bn.F32) == 0  # V % 8
     assert bn.workspace_bytes(bn.OP_VERIFY, 4, 65, 1024, 16, bn.F32) == 0  # K > 64
     assert bn.workspace_bytes(9, 4, 4, 1024, 16, bn.F32) == 0
+    # calibration: status block, 256 x 256 fp64 losses, 256 x K x 15 x 3 fp64 bin sums
+    assert bn.workspace_bytes(bn.OP_CALIB, 1000, 5, 0, 0, 0) == 256 + 256 * 256 * 8 + 256 * 5 * 15 * 3 * 8
+    assert bn.workspace_bytes(bn.OP_CALIB, 1000, 65, 0, 0, 0) == 0
 
 
 def test_null_pointers_rejected_before_any_device_call(lib):
@@ -54,6 +57,7 @@ def test_null_pointers_rejected_before_any_device_call(lib):
     assert lib.dspark_verify(p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
     assert lib.dspark_draft_logits(p, p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, p, p, 0, p) == -1
     assert lib.dspark_draft_pick(p, p, p, 4, 4, 1024, 0, 1, 0, 1, p, p, p, p, 0, p) == -1
+    assert lib.dspark_sts_fit(p, p, 100, 5, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_prefix_schedule(p, p, p, 0.0, 4, 4, 0, 0.0, p, p, p, 0, p) == -1
     assert lib.dspark_read_status(p, p, None, None) == -1
     assert lib.dspark_clear_status(p, p) == -1
