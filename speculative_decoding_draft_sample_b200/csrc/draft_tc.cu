@@ -99,10 +99,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t par) {
 }
 
 // L2 eviction policies: W is re-read by every draft position (keep it), base
-// and d stream through once per position (let them go first).
+// streams through once per position (let it go first).
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 __device__ __forceinline__ uint64_t policy_evict_first() {
@@ -460,7 +465,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc = (valid && p.bias_scale) ? p.bias_scale[b] : 1.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool elected = (warp == 4 + 4 * h) && lane == 0;
-    const uint64_t pol_d = policy_evict_first();
+    // d keeps the normal L2 priority: the sampler re-reads one 256-entry
+    // chunk of every row right after the position ends
+    const uint64_t pol_d = policy_evict_normal();
     bool miss = false;
     bool aborted = false;
     const bool leader = warp == 4 && lane == 0;
