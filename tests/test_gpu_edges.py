@@ -206,3 +206,31 @@ def test_schedule_on_side_stream_matches_one_stream(cuda_ok):
     assert a.status() == (0, -1) and b.status() == (0, -1)
     for name in ("x", "d", "q_tok", "cut", "survival", "accepted", "out", "n_emit"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
+
+
+def test_round_replayed_as_a_cuda_graph_matches_eager(cuda_ok):
+    """The round captured as a CUDA graph (the one-launch draft kernel with its
+    barrier-counter memset, the schedule on a forked side stream, verify) gives
+    the eager round's outputs on every replay."""
+    w = _small(B=150, V=8192, greedy_frac=0.2)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    eager = SpecRound(w.B, w.K, w.V, w.r)
+    eager.run(dev, SEED, 9)
+    torch.cuda.synchronize()
+    rnd = SpecRound(w.B, w.K, w.V, w.r)
+    main, side = torch.cuda.Stream(), torch.cuda.Stream()
+    with torch.cuda.stream(main):
+        rnd.run(dev, SEED, 9, stream=main, side_stream=side)  # warm-up outside capture
+        main.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=main):
+            rnd.run(dev, SEED, 9, stream=main, side_stream=side)
+        for _ in range(3):
+            rnd.out.fill_(-9)
+            g.replay()
+            main.synchronize()
+            for name in ("x", "d", "q_tok", "cut", "accepted", "out", "n_emit"):
+                assert torch.equal(getattr(rnd, name), getattr(eager, name)), name
+    assert rnd.status() == (0, -1)
+    del g
