@@ -761,19 +761,12 @@ int verify_cluster_size(int B, int V, int dtype, int num_sms) {
   return C;
 }
 
-size_t verify_smem_bytes(int V, int dtype, int C, int* slice, size_t* slice_padded) {
-  (void)dtype;
-  int s = (V + C - 1) / C;
-  s = (s + 7) & ~7;
-  if (slice) *slice = s;
-  if (slice_padded) *slice_padded = 0;
-  return 0;  // the 16 KB ring and the bookkeeping are static shared memory
-}
+// Vocabulary entries per CTA: an equal share, rounded up to a multiple of 8
+// (every slice starts on a 16-byte boundary).
+static int verify_slice(int V, int C) { return ((V + C - 1) / C + 7) & ~7; }
 
 cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s) {
-  size_t padded = 0;
-  const size_t sm = verify_smem_bytes(a.V, a.dtype, C, &a.slice, &padded);
-  a.slice_bytes_padded = padded;
+  a.slice = verify_slice(a.V, C);
   auto kern = (a.dtype == DSPARK_F32) ? verify_kernel<DSPARK_F32> : verify_kernel<DSPARK_BF16>;
   if (C > 8) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -782,7 +775,7 @@ cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.B * C));
   cfg.blockDim = dim3(kVThreads);
-  cfg.dynamicSmemBytes = sm;
+  cfg.dynamicSmemBytes = 0;  // the ring and the bookkeeping are static shared memory
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;

@@ -19,13 +19,10 @@ struct VerifyArgs {
   int32_t* n_emit;        // [B]
   Status* status;
   int slice;              // vocabulary entries per CTA (multiple of 8)
-  size_t slice_bytes_padded;
 };
 
 // CTAs per request (the cluster size) for this batch shape.
 int verify_cluster_size(int B, int V, int dtype, int num_sms);
-// Dynamic shared memory of one CTA; also returns the slice length and its padded bytes.
-size_t verify_smem_bytes(int V, int dtype, int C, int* slice, size_t* slice_padded);
 cudaError_t verify_launch(VerifyArgs a, int C, cudaStream_t s);
 
 }  // namespace dspark
