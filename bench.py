@@ -99,22 +99,33 @@ class Clocks:
                 "samples": len(self.samples), "source": "NVML every 2 ms over the timed region"}
 
 
-def profiled_traffic(kernel_file: str, summary: str):
-    """DRAM bytes per launch from a committed ncu summary, or None when the
-    kernel's source changed after the counters were taken."""
+# sources the draft kernel compiles from (its counters are valid while they hash the same)
+DRAFT_KERNEL_SOURCES = ("draft_tc.cu", "draft_tc.cuh", "draft.cuh", "sample_warp.cuh", "common.cuh")
+
+
+def sources_sha256(files) -> str:
     import hashlib
-    src = os.path.join(ROOT, "speculative_decoding_draft_sample_b200", "csrc", kernel_file)
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "speculative_decoding_draft_sample_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def profiled_traffic(kernel_files, summary: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel's sources changed after the counters were taken."""
     path = os.path.join(ROOT, "profiles", summary)
-    if not (os.path.exists(src) and os.path.exists(path)):
+    if not os.path.exists(path):
         return None, "no ncu summary committed"
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = sources_sha256(kernel_files)
     fields = {}
     for line in open(path):
         if ":" in line:
             k, v = line.split(":", 1)
             fields[k.strip()] = v.strip()
     if fields.get("source_sha256") != sha:
-        return None, "kernel source changed since the ncu capture"
+        return None, "kernel sources changed since the ncu capture"
     try:
         return float(fields["dram_bytes_per_launch"]), "profiles/" + summary
     except (KeyError, ValueError):
@@ -331,14 +342,15 @@ def main():
     with torch.cuda.stream(stream):
         ms_draft = time_region(lambda: bn.draft_sample(
             dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], dev["temp"],
-            wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream),
-            stream, 10)
+            wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream,
+            q_norm=rnd.q_norm), stream, 10)
         ms_sched = time_region(lambda: bn.prefix_schedule(
             dev["conf_logit"], dev["pos_temp"], dev["step_cost"], dev["fixed_cost"], bn.CUT_COST,
             0.0, rnd.cut, rnd.survival, rnd.ws, stream), stream, 20)
         ms_verify = time_region(lambda: bn.verify(
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
-            round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream), stream, 20)
+            round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream, q_norm=rnd.q_norm),
+            stream, 20)
 
     # verify's algorithmic bytes: target rows 0..a_b of every request, plus the
     # draft row a_b of every request rejected before its cut
@@ -371,7 +383,7 @@ def main():
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
     in_bytes = (w.B * (w.K + 1) * w.V + w.B * w.K * w.V + 2 * w.V * w.r) * s_bytes
-    traffic, traffic_src = profiled_traffic("draft_tc.cu", "draft_logits_tc_dspark5.txt")
+    traffic, traffic_src = profiled_traffic(DRAFT_KERNEL_SOURCES, "draft_logits_tc_dspark5.txt")
     if w.name != wl.DSPARK5.name:
         traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload only"
     roof = {"kernel": "draft_logits_tc (dspark_draft_sample: all K positions in one launch)",

@@ -113,6 +113,10 @@ size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype);
  *   d          [B, K, V] dtype out  stored draft logits (verification uses them)
  *   q_lse      [B, K] f32  out   log normaliser of d/temp
  *   q_tok      [B, K] f32  out   draft probability of each drafted token
+ *   q_norm     [B, K, 2] f32 out or NULL: the draw's normaliser as (m, s) with
+ *                                z = d log2(e) / temp, m = max z, s = sum 2^(z - m)
+ *                                ((max d, 1) for greedy rows); dspark_verify
+ *                                takes it to skip recomputing it
  * Limits: 1 <= B <= 65535, 1 <= K <= 64, 8 <= V < 2^24, 1 <= r <= 1024;
  * bf16 additionally needs r % 16 == 0.
  */
@@ -120,8 +124,8 @@ int dspark_draft_sample(const void* base, const void* U, const void* W,
                         const float* bias_scale, const int32_t* last_tok,
                         const float* temp, int B, int K, int V, int r, int dtype,
                         uint64_t seed, uint64_t round_id, int32_t* x, void* d,
-                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
-                        dspark_stream_t stream);
+                        float* q_lse, float* q_tok, float* q_norm, void* ws,
+                        size_t ws_bytes, dspark_stream_t stream);
 
 /*
  * The two halves of one draft position of dspark_draft_sample, for callers
@@ -137,7 +141,8 @@ int dspark_draft_sample(const void* base, const void* U, const void* W,
  *   x[b, k-2] for k >= 2 (so x[:, k-2] must hold position k-1's tokens), and
  *   the per-(request, 256-entry chunk) softmax partials of d/temp, kept in the
  *   workspace for the pick that follows. Arguments as for dspark_draft_sample.
- * dspark_draft_pick(k): x[:, k-1], q_lse[:, k-1], q_tok[:, k-1] from
+ * dspark_draft_pick(k): x[:, k-1], q_lse[:, k-1], q_tok[:, k-1] (and q_norm
+ *   when not NULL) from
  *   d[:, k-1, :] and the workspace partials that dspark_draft_logits(k) left
  *   (the workspace must not be used by another call in between). last_tok is
  *   read only to report a bad token at k = 1.
@@ -154,7 +159,7 @@ int dspark_draft_logits(const void* base, const void* U, const void* W,
 int dspark_draft_pick(const void* d, const int32_t* last_tok, const float* temp,
                       int B, int K, int V, int dtype, uint64_t seed,
                       uint64_t round_id, int k, int32_t* x, float* q_lse,
-                      float* q_tok, void* ws, size_t ws_bytes,
+                      float* q_tok, float* q_norm, void* ws, size_t ws_bytes,
                       dspark_stream_t stream);
 
 /*
@@ -208,11 +213,16 @@ int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp,
  *
  *   target [B, K+1, V] dtype, d [B, K, V] dtype, x [B, K] i32,
  *   q_tok [B, K] f32, cut [B] i32 or NULL (all K), temp [B] f32
+ *   q_norm [B, K, 2] f32 or NULL: the draft rows' normalisers as written by
+ *     dspark_draft_sample; with it a rejected request's residual starts at
+ *     once, without it the draft row's normaliser is recomputed (one more pass
+ *     over draft row a). The two agree up to fp32 summation order.
  *   accepted [B] i32 out, out [B, K+1] i32 out, n_emit [B] i32 out
  * Limits: 1 <= B <= 65535, 1 <= K <= 64, 8 <= V < 2^24.
  */
 int dspark_verify(const void* target, const void* d, const int32_t* x,
-                  const float* q_tok, const int32_t* cut, const float* temp,
+                  const float* q_tok, const float* q_norm, const int32_t* cut,
+                  const float* temp,
                   int B, int K, int V, int dtype, uint64_t seed,
                   uint64_t round_id, int32_t* accepted, int32_t* out,
                   int32_t* n_emit, void* ws, size_t ws_bytes,

@@ -34,14 +34,14 @@ _f = ctypes.c_float
 SIGNATURES = {
     "dspark_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i]),
     "dspark_draft_sample": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
-                                 _p, _p, _p, _p, _p, _sz, _p]),
+                                 _p, _p, _p, _p, _p, _p, _sz, _p]),
     "dspark_prefix_schedule": (_i, [_p, _p, _p, _f, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
-    "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
+    "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
                            _p, _sz, _p]),
     "dspark_draft_logits": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p,
                                  _sz, _p]),
-    "dspark_draft_pick": (_i, [_p, _p, _p, _i, _i, _i, _i, _u64, _u64, _i, _p, _p, _p, _p, _sz,
-                               _p]),
+    "dspark_draft_pick": (_i, [_p, _p, _p, _i, _i, _i, _i, _u64, _u64, _i, _p, _p, _p, _p, _p,
+                               _sz, _p]),
     "dspark_draft_sample_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
                                         _p, _p, _p, _p, _p, _p]),
     "dspark_sts_fit": (_i, [_p, _p, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
@@ -114,8 +114,9 @@ def version() -> int:
 
 
 def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: int,
-                 x, d, q_lse, q_tok, ws, stream=None) -> None:
-    """dspark_draft_sample: base [B,K,V], U [V,r], W [r,V] -> x, d, q_lse, q_tok."""
+                 x, d, q_lse, q_tok, ws, stream=None, q_norm=None) -> None:
+    """dspark_draft_sample: base [B,K,V], U [V,r], W [r,V] -> x, d, q_lse, q_tok
+    (and q_norm [B,K,2] when given)."""
     B, K, V = base.shape
     r = U.shape[1]
     dt = _dtype_code(base)
@@ -124,8 +125,8 @@ def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: in
         _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
         _ptr(temp, "temp", torch.float32), B, K, V, r, dt, seed, round_id,
         _ptr(x, "x", torch.int32), _ptr(d, "d", base.dtype), _ptr(q_lse, "q_lse", torch.float32),
-        _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
-        _stream(stream))
+        _ptr(q_tok, "q_tok", torch.float32), _ptr(q_norm, "q_norm", torch.float32), _ptr(ws, "ws"),
+        ws.numel() * ws.element_size(), _stream(stream))
     _check(rc, "dspark_draft_sample")
 
 
@@ -144,14 +145,15 @@ def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, strea
 
 
 def draft_pick(d, last_tok, temp, seed: int, round_id: int, k: int, x, q_lse, q_tok, ws,
-               stream=None) -> None:
+               stream=None, q_norm=None) -> None:
     """dspark_draft_pick: position k's token, q_lse and q_tok from d[:, k-1]."""
     B, K, V = d.shape
     rc = lib().dspark_draft_pick(
         _ptr(d, "d"), _ptr(last_tok, "last_tok", torch.int32), _ptr(temp, "temp", torch.float32),
         B, K, V, _dtype_code(d), seed, round_id, int(k), _ptr(x, "x", torch.int32),
-        _ptr(q_lse, "q_lse", torch.float32), _ptr(q_tok, "q_tok", torch.float32), _ptr(ws, "ws"),
-        ws.numel() * ws.element_size(), _stream(stream))
+        _ptr(q_lse, "q_lse", torch.float32), _ptr(q_tok, "q_tok", torch.float32),
+        _ptr(q_norm, "q_norm", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
+        _stream(stream))
     _check(rc, "dspark_draft_pick")
 
 
@@ -185,13 +187,14 @@ def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: in
 
 
 def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out, n_emit,
-           ws, stream=None) -> None:
+           ws, stream=None, q_norm=None) -> None:
     """dspark_verify: target [B,K+1,V], d [B,K,V], x, q_tok [B,K], cut [B] -> accepted, out, n_emit."""
     B, K1, V = target.shape
     dt = _dtype_code(target)
     rc = lib().dspark_verify(
         _ptr(target, "target"), _ptr(d, "d", target.dtype), _ptr(x, "x", torch.int32),
-        _ptr(q_tok, "q_tok", torch.float32), _ptr(cut, "cut", torch.int32),
+        _ptr(q_tok, "q_tok", torch.float32), _ptr(q_norm, "q_norm", torch.float32),
+        _ptr(cut, "cut", torch.int32),
         _ptr(temp, "temp", torch.float32), B, K1 - 1, V, dt, seed, round_id,
         _ptr(accepted, "accepted", torch.int32), _ptr(out, "out", torch.int32),
         _ptr(n_emit, "n_emit", torch.int32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),

@@ -14,7 +14,7 @@ using namespace dspark;
 
 namespace {
 
-constexpr int kAbiVersion = (1 << 16) | 0;
+constexpr int kAbiVersion = (2 << 16) | 0;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -108,7 +108,7 @@ namespace {
 int draft_prepare(DraftArgs& a, int* sms, bool logits, bool pick, const void* base, const void* U,
                   const void* W, const float* bias_scale, const int32_t* last_tok, const float* temp,
                   int B, int K, int V, int r, int dtype, uint64_t seed, uint64_t round_id, int32_t* x,
-                  void* d, float* q_lse, float* q_tok, void* ws, size_t ws_bytes) {
+                  void* d, float* q_lse, float* q_tok, float* q_norm, void* ws, size_t ws_bytes) {
   if (!last_tok || !temp || !x || !d || !ws) return DSPARK_ERR_INVALID_ARG;
   if (logits && (!base || !U || !W)) return DSPARK_ERR_INVALID_ARG;
   if (pick && (!q_lse || !q_tok)) return DSPARK_ERR_INVALID_ARG;
@@ -136,6 +136,7 @@ int draft_prepare(DraftArgs& a, int* sms, bool logits, bool pick, const void* ba
   a.d = d;
   a.q_lse = q_lse;
   a.q_tok = q_tok;
+  a.q_norm = reinterpret_cast<float2*>(q_norm);
   a.status = static_cast<Status*>(ws);
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   a.nchunk = nchunks(V);
@@ -153,12 +154,12 @@ extern "C" {
 int dspark_draft_sample(const void* base, const void* U, const void* W, const float* bias_scale,
                         const int32_t* last_tok, const float* temp, int B, int K, int V, int r,
                         int dtype, uint64_t seed, uint64_t round_id, int32_t* x, void* d,
-                        float* q_lse, float* q_tok, void* ws, size_t ws_bytes,
+                        float* q_lse, float* q_tok, float* q_norm, void* ws, size_t ws_bytes,
                         dspark_stream_t stream) {
   DraftArgs a;
   int sms = 0;
   if (int e = draft_prepare(a, &sms, true, true, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
-                            dtype, seed, round_id, x, d, q_lse, q_tok, ws, ws_bytes))
+                            dtype, seed, round_id, x, d, q_lse, q_tok, q_norm, ws, ws_bytes))
     return e;
   cudaStream_t s = (cudaStream_t)stream;
   // one cooperative launch for the whole block when the tensor-core path
@@ -181,19 +182,20 @@ int dspark_draft_logits(const void* base, const void* U, const void* W, const fl
   DraftArgs a;
   int sms = 0;
   if (int e = draft_prepare(a, &sms, true, false, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
-                            dtype, 0, 0, const_cast<int32_t*>(x), d, nullptr, nullptr, ws, ws_bytes))
+                            dtype, 0, 0, const_cast<int32_t*>(x), d, nullptr, nullptr, nullptr, ws,
+                            ws_bytes))
     return e;
   return cuda_status(launch_logits(a, k, sms, (cudaStream_t)stream));
 }
 
 int dspark_draft_pick(const void* d, const int32_t* last_tok, const float* temp, int B, int K, int V,
                       int dtype, uint64_t seed, uint64_t round_id, int k, int32_t* x, float* q_lse,
-                      float* q_tok, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+                      float* q_tok, float* q_norm, void* ws, size_t ws_bytes, dspark_stream_t stream) {
   if (k < 1 || k > K) return DSPARK_ERR_INVALID_ARG;
   DraftArgs a;
   if (int e = draft_prepare(a, nullptr, false, true, nullptr, nullptr, nullptr, nullptr, last_tok, temp,
                             B, K, V, 16, dtype, seed, round_id, x, const_cast<void*>(d), q_lse, q_tok,
-                            ws, ws_bytes))
+                            q_norm, ws, ws_bytes))
     return e;
   return cuda_status(draft_sample_launch(a, k, (cudaStream_t)stream));
 }
@@ -227,6 +229,7 @@ int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp, const
 }
 
 int dspark_verify(const void* target, const void* d, const int32_t* x, const float* q_tok,
+                  const float* q_norm,
                   const int32_t* cut, const float* temp, int B, int K, int V, int dtype,
                   uint64_t seed, uint64_t round_id, int32_t* accepted, int32_t* out,
                   int32_t* n_emit, void* ws, size_t ws_bytes, dspark_stream_t stream) {
@@ -243,6 +246,7 @@ int dspark_verify(const void* target, const void* d, const int32_t* x, const flo
   a.d = d;
   a.x = x;
   a.q_tok = q_tok;
+  a.q_norm = reinterpret_cast<const float2*>(q_norm);
   a.cut = cut;
   a.temp = temp;
   a.B = B;

@@ -22,6 +22,7 @@ struct DraftArgs {
   void* d;                 // [B, K, V]
   float* q_lse;            // [B, K]
   float* q_tok;            // [B, K]
+  float2* q_norm;          // [B, K] (max z, sum 2^(z - max)) of z = d log2(e) / temp, or null
   float2* partials;        // [B, nchunk] in the workspace
   int nchunk;
   Status* status;

@@ -115,6 +115,7 @@ extern "C" int dspark_draft_sample_static(const void* base, const void* U, const
   a.d = d;
   a.q_lse = q_lse;
   a.q_tok = q_tok;
+  a.q_norm = nullptr;
   a.status = static_cast<Status*>(scratch);
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(scratch) + kStatusBytes);
   a.nchunk = nchunk;

@@ -66,6 +66,7 @@ __device__ __forceinline__ void sample_row_warp(const DraftArgs& a, int b, int k
       a.x[out_i] = i;
       a.q_tok[out_i] = 1.f;
       a.q_lse[out_i] = mv;
+      if (a.q_norm) a.q_norm[out_i] = make_float2(mv, 1.f);
       prefetch_u_row<DT>(a, i, k);
     }
     return;
@@ -106,6 +107,7 @@ __device__ __forceinline__ void sample_row_warp(const DraftArgs& a, int b, int k
       a.x[out_i] = 0;
       a.q_tok[out_i] = 0.f;
       a.q_lse[out_i] = NAN;
+      if (a.q_norm) a.q_norm[out_i] = make_float2(NAN, 0.f);
     }
     return;
   }
@@ -214,10 +216,12 @@ __device__ __forceinline__ void sample_row_warp(const DraftArgs& a, int b, int k
       a.x[out_i] = 0;
       a.q_tok[out_i] = 0.f;
       a.q_lse[out_i] = NAN;
+      if (a.q_norm) a.q_norm[out_i] = make_float2(NAN, 0.f);
     } else {
       a.x[out_i] = v0 + tj;
       a.q_tok[out_i] = wt / Z;
       a.q_lse[out_i] = M * 0.69314718055994530942f + logf(Z);
+      if (a.q_norm) a.q_norm[out_i] = make_float2(M, Z);
       prefetch_u_row<DT>(a, v0 + tj, k);
     }
   }

@@ -677,9 +677,16 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
     // (q = softmax(d / temp), its normaliser recomputed here)
     const T* trow = target + (long long)acc * V + c.lo;
     const T* drow = drow0 + (long long)acc * V + c.lo;
-    const float2 mq = c.row_stats(drow, cs);
-    c.gather(Exch{mq.x, mq.y, 0.f, 0});
-    const float2 MZq = combine_ranks(got, c.C);
+    // the draft row's normaliser: from the draw that produced it when the
+    // caller passes it on, else one more pass over the draft row
+    float2 MZq;
+    if (a.q_norm) {
+      MZq = a.q_norm[(long long)b * K + acc];
+    } else {
+      const float2 mq = c.row_stats(drow, cs);
+      c.gather(Exch{mq.x, mq.y, 0.f, 0});
+      MZq = combine_ranks(got, c.C);
+    }
     const float Mq = MZq.x, iZ = 1.f / Z, iZq = 1.f / MZq.y;
     auto resid = [&](float tv, float dv) {
       const float pp = ex2(fmaf(tv, cs, -M)) * iZ;

@@ -10,6 +10,7 @@ struct VerifyArgs {
   const void* d;          // [B, K, V]
   const int32_t* x;       // [B, K]
   const float* q_tok;     // [B, K]
+  const float2* q_norm;   // [B, K] draft-row normalisers (max z, sum 2^(z - max)) or null
   const int32_t* cut;     // [B] or null
   const float* temp;      // [B]
   int B, K, V, dtype;

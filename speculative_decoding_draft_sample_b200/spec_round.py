@@ -27,6 +27,7 @@ class SpecRound:
         self.d = torch.empty((B, K, V), dtype=dtype, device=dev)
         self.q_lse = torch.empty((B, K), **f32)
         self.q_tok = torch.empty((B, K), **f32)
+        self.q_norm = torch.empty((B, K, 2), **f32)  # the draws' normalisers, for verify
         self.cut = torch.empty((B,), **i32)
         self.survival = torch.empty((B, K), **f32)
         self.accepted = torch.empty((B,), **i32)
@@ -64,13 +65,13 @@ class SpecRound:
             join.record(side_stream)
         bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
                         inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
-                        self.ws, main)
+                        self.ws, main, q_norm=self.q_norm)
         if side_stream is None:
             schedule(main)
         else:
             main.wait_event(join)
         bn.verify(inp["target"], self.d, self.x, self.q_tok, self.cut, inp["temp"], seed,
-                  round_id, self.accepted, self.out, self.n_emit, self.ws, main)
+                  round_id, self.accepted, self.out, self.n_emit, self.ws, main, q_norm=self.q_norm)
 
     def status(self, stream=None):
         return bn.read_status(self.ws, stream)

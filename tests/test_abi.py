@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert bn.version() >> 16 == 1
+    assert bn.version() >> 16 == 2
     assert lib.dspark_status_string(0) == b"ok"
     assert b"workspace" in lib.dspark_status_string(-4)
 
@@ -53,10 +53,10 @@ def test_workspace_sizes(lib):
 
 def test_null_pointers_rejected_before_any_device_call(lib):
     p = ctypes.c_void_p(0)
-    assert lib.dspark_draft_sample(p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p, p, 0, p) == -1
-    assert lib.dspark_verify(p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
+    assert lib.dspark_draft_sample(p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p, p, p, 0, p) == -1
+    assert lib.dspark_verify(p, p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
     assert lib.dspark_draft_logits(p, p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, p, p, 0, p) == -1
-    assert lib.dspark_draft_pick(p, p, p, 4, 4, 1024, 0, 1, 0, 1, p, p, p, p, 0, p) == -1
+    assert lib.dspark_draft_pick(p, p, p, 4, 4, 1024, 0, 1, 0, 1, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_sts_fit(p, p, 100, 5, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_prefix_schedule(p, p, p, 0.0, 4, 4, 0, 0.0, p, p, p, 0, p) == -1
     assert lib.dspark_read_status(p, p, None, None) == -1

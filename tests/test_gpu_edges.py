@@ -234,3 +234,31 @@ def test_round_replayed_as_a_cuda_graph_matches_eager(cuda_ok):
                 assert torch.equal(getattr(rnd, name), getattr(eager, name)), name
     assert rnd.status() == (0, -1)
     del g
+
+
+def test_verify_with_and_without_the_draft_normalisers(cuda_ok):
+    """dspark_verify given the draws' normalisers (q_norm) and recomputing them
+    (NULL) take the same decisions and emit the same tokens."""
+    w = _small(B=160, V=8192, independent_frac=0.3, greedy_frac=0.1)
+    inp = wl.generate(w)
+    dev = to_device(inp)
+    rnd = SpecRound(w.B, w.K, w.V, w.r)
+    rnd.run(dev, SEED, 4)
+    acc2, out2, n2 = torch.empty_like(rnd.accepted), torch.empty_like(rnd.out), torch.empty_like(rnd.n_emit)
+    bn.verify(dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], SEED, 4, acc2, out2, n2,
+              rnd.ws)
+    torch.cuda.synchronize()
+    assert rnd.status() == (0, -1)
+    assert (rnd.accepted < rnd.cut).any()  # some residual draws happen
+    assert torch.equal(acc2, rnd.accepted) and torch.equal(out2, rnd.out) and torch.equal(n2, rnd.n_emit)
+    # the normalisers are those of the stored draft logits: q_tok = 2^(d_x cs - m) / s
+    qn = rnd.q_norm.cpu().double().numpy()
+    d = rnd.d.float().cpu().double().numpy()
+    x = rnd.x.cpu().numpy()
+    tau = dev["temp"].cpu().double().numpy()
+    for b in range(0, w.B, 17):
+        if tau[b] > 0:
+            cs = 1.4426950408889634 / tau[b]
+            for k in range(w.K):
+                q = 2.0 ** (d[b, k, x[b, k]] * cs - qn[b, k, 0]) / qn[b, k, 1]
+                assert abs(q - rnd.q_tok[b, k].item()) <= 1e-5 * max(q, 1e-30)
