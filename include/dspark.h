@@ -268,7 +268,8 @@ int dspark_sts_fit(const float* conf_logit, const uint8_t* survived, int N, int 
  * cudaMalloc's implicit synchronisation have no way to provide one.
  *
  * Same arguments, computation and results as dspark_draft_sample, without
- * ws/ws_bytes. The scratch is a fixed 8 MiB array inside the library's device
+ * ws/ws_bytes and without the optional q_norm output (dspark_verify then
+ * recomputes the draft rows' normalisers). The scratch is a fixed 8 MiB array inside the library's device
  * image, held on every GPU that loads the library until the process exits; the
  * call allocates and frees nothing. Its device address is looked up once per
  * device, by the first call made while that device is current, so that first
