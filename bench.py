@@ -38,6 +38,9 @@ UNIT = "rounds/s"
 L2_BYTES = 126 * 1024 * 1024
 
 
+CUT_MODES = {"cost": bn.CUT_COST, "threshold": bn.CUT_THRESHOLD, "none": bn.CUT_NONE}
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -145,7 +148,8 @@ def time_region(fn, stream, iters: int) -> float:
     return e0.elapsed_time(e1) / iters
 
 
-def cpu_baseline(w: wl.Workload, inp_small, n_req: int, round_id: int):
+def cpu_baseline(w: wl.Workload, inp_small, n_req: int, round_id: int, mode: int = bn.CUT_COST,
+                 threshold: float = 0.0):
     """The fp64 oracle on a bounded sample of the round (n_req requests)."""
     from oracle import dspark as o
     try:
@@ -166,7 +170,7 @@ def cpu_baseline(w: wl.Workload, inp_small, n_req: int, round_id: int):
               step_cost=np.asarray(inp_small["step_cost"], np.float64),
               fixed_cost=float(inp_small["fixed_cost"]), dtype=w.dtype, request_ids=rid)
     t0 = time.perf_counter()
-    r = o.run_round(oi, wl.PHILOX_SEED, round_id)
+    r = o.run_round(oi, wl.PHILOX_SEED, round_id, mode, threshold)
     dt = time.perf_counter() - t0
     rounds = n_req / w.B
     return dict(value=rounds / dt, unit=UNIT, cores=int(cores), kind="oracle",
@@ -181,19 +185,22 @@ def reference_arm(args, w: wl.Workload):
         return
     small = wl.small_inputs(w)
     n_req = 4
+    mode = CUT_MODES[args.cut]
+    threshold = args.threshold if mode == bn.CUT_THRESHOLD else 0.0
     for i in range(args.warmup):
-        cpu_baseline(w, small, 1, 1000 + i)
+        cpu_baseline(w, small, 1, 1000 + i, mode, threshold)
     secs = 0.0
     last = None
     for i in range(args.steps):
-        last = cpu_baseline(w, small, n_req, i)
+        last = cpu_baseline(w, small, n_req, i, mode, threshold)
         secs += last["seconds"]
     value = args.steps * (n_req / w.B) / secs
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r},
+            "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
+                       "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else "")},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
                              "sample": last["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -263,6 +270,11 @@ def main():
                     help="prefix schedule only: mean cut and time as the batch grows")
     ap.add_argument("--calib", type=int, default=0, metavar="N",
                     help="Sequential Temperature Scaling of N synthetic samples (K = 5): time and ECE")
+    ap.add_argument("--cut", default="cost", choices=sorted(CUT_MODES),
+                    help="prefix schedule: early-stopping cost rule (default), static survival "
+                         "threshold, or none (every request verifies all K drafts)")
+    ap.add_argument("--threshold", type=float, default=0.5,
+                    help="survival threshold of --cut threshold")
     args = ap.parse_args()
     if args.load_sweep:
         load_sweep()
@@ -287,8 +299,11 @@ def main():
     side = torch.cuda.Stream()  # the prefix schedule runs here, beside the draft
     round_id = 0
 
+    mode = CUT_MODES[args.cut]
+    threshold = args.threshold if mode == bn.CUT_THRESHOLD else 0.0
+
     def step():
-        rnd.run(dev, wl.PHILOX_SEED, round_id, stream=stream, side_stream=side)
+        rnd.run(dev, wl.PHILOX_SEED, round_id, mode, threshold, stream=stream, side_stream=side)
 
     with torch.cuda.stream(stream):
         step()
@@ -345,8 +360,8 @@ def main():
             wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream,
             q_norm=rnd.q_norm), stream, 10)
         ms_sched = time_region(lambda: bn.prefix_schedule(
-            dev["conf_logit"], dev["pos_temp"], dev["step_cost"], dev["fixed_cost"], bn.CUT_COST,
-            0.0, rnd.cut, rnd.survival, rnd.ws, stream), stream, 20)
+            dev["conf_logit"], dev["pos_temp"], dev["step_cost"], dev["fixed_cost"], mode,
+            threshold, rnd.cut, rnd.survival, rnd.ws, stream), stream, 20)
         ms_verify = time_region(lambda: bn.verify(
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
             round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream, q_norm=rnd.q_norm),
@@ -374,18 +389,19 @@ def main():
     d2h = out_h.numel() * 4 + n_h.numel() * 4
     with torch.cuda.stream(stream):
         for _ in range(2):
-            run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, stream=stream,
-                     side_stream=side)
+            run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, mode, stream=stream,
+                     side_stream=side, threshold=threshold)
         replicas.barrier()
         e2e_steps = max(3, args.steps // 5)
         ms_e2e = time_region(lambda: run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h,
-                                              stream=stream, side_stream=side), stream, e2e_steps)
+                                              mode, stream=stream, side_stream=side,
+                                              threshold=threshold), stream, e2e_steps)
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
     in_bytes = (w.B * (w.K + 1) * w.V + w.B * w.K * w.V + 2 * w.V * w.r) * s_bytes
     traffic, traffic_src = profiled_traffic(DRAFT_KERNEL_SOURCES, "draft_logits_tc_dspark5.txt")
-    if w.name != wl.DSPARK5.name:
-        traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload only"
+    if w.name != wl.DSPARK5.name or mode != bn.CUT_COST:
+        traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload (cost cut) only"
     roof = {"kernel": "draft_logits_tc (dspark_draft_sample: all K positions in one launch)",
             "bound": "hbm", "achieved": draft_gbs, "peak": hbm, "unit": "GB/s",
             "frac": draft_gbs / hbm, "traffic": traffic, "traffic_source": traffic_src,
@@ -400,6 +416,7 @@ def main():
         "data": "synthetic (seeded Zipf+noise logits, random Markov factors)",
         "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
                    "global_batch": w.B * world, "parallelism": f"replicas{world}",
+                   "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else ""),
                    "l2": (f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2 (126 MB); not flushed"
                           if in_bytes > L2_BYTES else
                           f"inputs ({in_bytes / 1e6:.0f} MB) fit in L2 (126 MB); not flushed"),
@@ -419,7 +436,8 @@ def main():
         "gpu_launches": 3 * args.steps,
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name
+            and mode == bn.CUT_COST):
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), 128, 0).items()
                                 if k in ("value", "unit", "cores", "kind", "sample")}
     del graph  # released before the process group goes away

@@ -99,10 +99,11 @@ def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -
 
 def run_host(rnd: SpecRound, host: Dict[str, object], dev: Dict[str, object], seed: int,
              round_id: int, out_host: torch.Tensor, n_emit_host: torch.Tensor,
-             mode: int = bn.CUT_COST, stream=None, side_stream=None) -> None:
+             mode: int = bn.CUT_COST, stream=None, side_stream=None,
+             threshold: float = 0.0) -> None:
     """End to end from pinned host buffers: H2D copies, the round, D2H of the tokens."""
     for k in DEVICE_KEYS:
         dev[k].copy_(host[k], non_blocking=True)
-    rnd.run(dev, seed, round_id, mode, stream=stream, side_stream=side_stream)
+    rnd.run(dev, seed, round_id, mode, threshold, stream=stream, side_stream=side_stream)
     out_host.copy_(rnd.out, non_blocking=True)
     n_emit_host.copy_(rnd.n_emit, non_blocking=True)
