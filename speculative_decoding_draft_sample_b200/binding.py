@@ -87,16 +87,35 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise DSparkError(f"unsupported logit dtype {t.dtype}")
 
 
-def _ptr(t: Optional[torch.Tensor], name: str, dtype=None) -> Optional[int]:
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, shape=None,
+         device=None) -> Optional[int]:
+    """The tensor's device pointer after checking it against the call's shapes.
+
+    The library sees only pointers and the sizes B, K, V, r; a tensor smaller
+    than those sizes imply would be read or written past its end on the device,
+    so every tensor's shape is checked here (`shape`), as are its dtype,
+    layout and device (`device`: the device of the call's first tensor).
+    """
     if t is None:
         return None
-    if not t.is_cuda:
-        raise DSparkError(f"{name} must be a CUDA tensor")
-    if not t.is_contiguous():
-        raise DSparkError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise DSparkError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise DSparkError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise DSparkError(f"{name} must be contiguous")
+    if device is None:
+        if not t.is_cuda:
+            raise DSparkError(f"{name} must be a CUDA tensor")
+    elif t.device != device:
+        raise DSparkError(f"{name} is on {t.device}, the call's tensors on {device}")
     return t.data_ptr()
+
+
+def _on_gpu(device: torch.device) -> None:
+    """Every tensor of a call is on `device` (checked by _ptr); it must be a GPU."""
+    if device.type != "cuda":
+        raise DSparkError(f"the call's tensors must be CUDA tensors, not on {device}")
 
 
 def _stream(stream) -> Optional[int]:
@@ -120,13 +139,18 @@ def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: in
     B, K, V = base.shape
     r = U.shape[1]
     dt = _dtype_code(base)
-    rc = lib().dspark_draft_sample(
-        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
-        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
-        _ptr(temp, "temp", torch.float32), B, K, V, r, dt, seed, round_id,
-        _ptr(x, "x", torch.int32), _ptr(d, "d", base.dtype), _ptr(q_lse, "q_lse", torch.float32),
-        _ptr(q_tok, "q_tok", torch.float32), _ptr(q_norm, "q_norm", torch.float32), _ptr(ws, "ws"),
-        ws.numel() * ws.element_size(), _stream(stream))
+    dev, f32, i32 = base.device, torch.float32, torch.int32
+    args = (
+        _ptr(base, "base", None, (B, K, V), dev), _ptr(U, "U", base.dtype, (V, r), dev),
+        _ptr(W, "W", base.dtype, (r, V), dev), _ptr(bias_scale, "bias_scale", f32, (B,), dev),
+        _ptr(last_tok, "last_tok", i32, (B,), dev), _ptr(temp, "temp", f32, (B,), dev),
+        B, K, V, r, dt, seed, round_id,
+        _ptr(x, "x", i32, (B, K), dev), _ptr(d, "d", base.dtype, (B, K, V), dev),
+        _ptr(q_lse, "q_lse", f32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
+        _ptr(q_norm, "q_norm", f32, (B, K, 2), dev), _ptr(ws, "ws", None, None, dev),
+        ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_draft_sample(*args, _stream(stream))
     _check(rc, "dspark_draft_sample")
 
 
@@ -136,11 +160,16 @@ def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, strea
     B, K, V = base.shape
     r = U.shape[1]
     dt = _dtype_code(base)
-    rc = lib().dspark_draft_logits(
-        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
-        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
-        _ptr(x, "x", torch.int32), _ptr(temp, "temp", torch.float32), B, K, V, r, dt, int(k),
-        _ptr(d, "d", base.dtype), _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    dev, f32, i32 = base.device, torch.float32, torch.int32
+    args = (
+        _ptr(base, "base", None, (B, K, V), dev), _ptr(U, "U", base.dtype, (V, r), dev),
+        _ptr(W, "W", base.dtype, (r, V), dev), _ptr(bias_scale, "bias_scale", f32, (B,), dev),
+        _ptr(last_tok, "last_tok", i32, (B,), dev), _ptr(x, "x", i32, (B, K), dev),
+        _ptr(temp, "temp", f32, (B,), dev), B, K, V, r, dt, int(k),
+        _ptr(d, "d", base.dtype, (B, K, V), dev), _ptr(ws, "ws", None, None, dev),
+        ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_draft_logits(*args, _stream(stream))
     _check(rc, "dspark_draft_logits")
 
 
@@ -148,12 +177,15 @@ def draft_pick(d, last_tok, temp, seed: int, round_id: int, k: int, x, q_lse, q_
                stream=None, q_norm=None) -> None:
     """dspark_draft_pick: position k's token, q_lse and q_tok from d[:, k-1]."""
     B, K, V = d.shape
-    rc = lib().dspark_draft_pick(
-        _ptr(d, "d"), _ptr(last_tok, "last_tok", torch.int32), _ptr(temp, "temp", torch.float32),
-        B, K, V, _dtype_code(d), seed, round_id, int(k), _ptr(x, "x", torch.int32),
-        _ptr(q_lse, "q_lse", torch.float32), _ptr(q_tok, "q_tok", torch.float32),
-        _ptr(q_norm, "q_norm", torch.float32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
-        _stream(stream))
+    dev, f32, i32 = d.device, torch.float32, torch.int32
+    args = (
+        _ptr(d, "d", None, (B, K, V), dev), _ptr(last_tok, "last_tok", i32, (B,), dev),
+        _ptr(temp, "temp", f32, (B,), dev), B, K, V, _dtype_code(d), seed, round_id, int(k),
+        _ptr(x, "x", i32, (B, K), dev), _ptr(q_lse, "q_lse", f32, (B, K), dev),
+        _ptr(q_tok, "q_tok", f32, (B, K), dev), _ptr(q_norm, "q_norm", f32, (B, K, 2), dev),
+        _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_draft_pick(*args, _stream(stream))
     _check(rc, "dspark_draft_pick")
 
 
@@ -164,13 +196,17 @@ def draft_sample_static(base, U, W, bias_scale, last_tok, temp, seed: int, round
     B, K, V = base.shape
     r = U.shape[1]
     dt = _dtype_code(base)
-    rc = lib().dspark_draft_sample_static(
-        _ptr(base, "base"), _ptr(U, "U", base.dtype), _ptr(W, "W", base.dtype),
-        _ptr(bias_scale, "bias_scale", torch.float32), _ptr(last_tok, "last_tok", torch.int32),
-        _ptr(temp, "temp", torch.float32), B, K, V, r, dt, seed, round_id,
-        _ptr(x, "x", torch.int32), _ptr(d, "d", base.dtype), _ptr(q_lse, "q_lse", torch.float32),
-        _ptr(q_tok, "q_tok", torch.float32), _ptr(status_out, "status_out", torch.int32),
-        _stream(stream))
+    dev, f32, i32 = base.device, torch.float32, torch.int32
+    args = (
+        _ptr(base, "base", None, (B, K, V), dev), _ptr(U, "U", base.dtype, (V, r), dev),
+        _ptr(W, "W", base.dtype, (r, V), dev), _ptr(bias_scale, "bias_scale", f32, (B,), dev),
+        _ptr(last_tok, "last_tok", i32, (B,), dev), _ptr(temp, "temp", f32, (B,), dev),
+        B, K, V, r, dt, seed, round_id,
+        _ptr(x, "x", i32, (B, K), dev), _ptr(d, "d", base.dtype, (B, K, V), dev),
+        _ptr(q_lse, "q_lse", f32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
+        _ptr(status_out, "status_out", i32, (2,), dev))
+    _on_gpu(dev)
+    rc = lib().dspark_draft_sample_static(*args, _stream(stream))
     _check(rc, "dspark_draft_sample_static")
 
 
@@ -178,11 +214,15 @@ def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: in
                     threshold: float, cut, survival, ws, stream=None) -> None:
     """dspark_prefix_schedule: conf_logit [B,K], pos_temp [K], step_cost [B(K+1)] -> cut, survival."""
     B, K = conf_logit.shape
-    rc = lib().dspark_prefix_schedule(
-        _ptr(conf_logit, "conf_logit", torch.float32), _ptr(pos_temp, "pos_temp", torch.float32),
-        _ptr(step_cost, "step_cost", torch.float32), float(fixed_cost), B, K, mode,
-        float(threshold), _ptr(cut, "cut", torch.int32), _ptr(survival, "survival", torch.float32),
-        _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    dev, f32 = conf_logit.device, torch.float32
+    args = (
+        _ptr(conf_logit, "conf_logit", f32, (B, K), dev), _ptr(pos_temp, "pos_temp", f32, (K,), dev),
+        _ptr(step_cost, "step_cost", f32, (B * (K + 1),), dev), float(fixed_cost), B, K, mode,
+        float(threshold), _ptr(cut, "cut", torch.int32, (B,), dev),
+        _ptr(survival, "survival", f32, (B, K), dev), _ptr(ws, "ws", None, None, dev),
+        ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_prefix_schedule(*args, _stream(stream))
     _check(rc, "dspark_prefix_schedule")
 
 
@@ -190,26 +230,34 @@ def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, o
            ws, stream=None, q_norm=None) -> None:
     """dspark_verify: target [B,K+1,V], d [B,K,V], x, q_tok [B,K], cut [B] -> accepted, out, n_emit."""
     B, K1, V = target.shape
+    K = K1 - 1
     dt = _dtype_code(target)
-    rc = lib().dspark_verify(
-        _ptr(target, "target"), _ptr(d, "d", target.dtype), _ptr(x, "x", torch.int32),
-        _ptr(q_tok, "q_tok", torch.float32), _ptr(q_norm, "q_norm", torch.float32),
-        _ptr(cut, "cut", torch.int32),
-        _ptr(temp, "temp", torch.float32), B, K1 - 1, V, dt, seed, round_id,
-        _ptr(accepted, "accepted", torch.int32), _ptr(out, "out", torch.int32),
-        _ptr(n_emit, "n_emit", torch.int32), _ptr(ws, "ws"), ws.numel() * ws.element_size(),
-        _stream(stream))
+    dev, f32, i32 = target.device, torch.float32, torch.int32
+    args = (
+        _ptr(target, "target", None, (B, K1, V), dev), _ptr(d, "d", target.dtype, (B, K, V), dev),
+        _ptr(x, "x", i32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
+        _ptr(q_norm, "q_norm", f32, (B, K, 2), dev), _ptr(cut, "cut", i32, (B,), dev),
+        _ptr(temp, "temp", f32, (B,), dev), B, K, V, dt, seed, round_id,
+        _ptr(accepted, "accepted", i32, (B,), dev), _ptr(out, "out", i32, (B, K1), dev),
+        _ptr(n_emit, "n_emit", i32, (B,), dev), _ptr(ws, "ws", None, None, dev),
+        ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_verify(*args, _stream(stream))
     _check(rc, "dspark_verify")
 
 
 def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, stream=None) -> None:
     """dspark_sts_fit: conf_logit [N,K] f32, survived [N,K] u8 -> T [K], index [K], ECE [K] x 2."""
     N, K = conf_logit.shape
-    rc = lib().dspark_sts_fit(
-        _ptr(conf_logit, "conf_logit", torch.float32), _ptr(survived, "survived", torch.uint8), N, K,
-        _ptr(T_out, "T_out", torch.float32), _ptr(index_out, "index_out", torch.int32),
-        _ptr(ece_before, "ece_before", torch.float32), _ptr(ece_after, "ece_after", torch.float32),
-        _ptr(ws, "ws"), ws.numel() * ws.element_size(), _stream(stream))
+    dev, f32 = conf_logit.device, torch.float32
+    args = (
+        _ptr(conf_logit, "conf_logit", f32, (N, K), dev),
+        _ptr(survived, "survived", torch.uint8, (N, K), dev), N, K,
+        _ptr(T_out, "T_out", f32, (K,), dev), _ptr(index_out, "index_out", torch.int32, (K,), dev),
+        _ptr(ece_before, "ece_before", f32, (K,), dev), _ptr(ece_after, "ece_after", f32, (K,), dev),
+        _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    rc = lib().dspark_sts_fit(*args, _stream(stream))
     _check(rc, "dspark_sts_fit")
 
 
