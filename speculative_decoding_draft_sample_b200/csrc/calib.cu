@@ -14,9 +14,9 @@
 // contiguous range of samples and thread t accumulates, in fp64 and in sample
 // order, the loss of grid temperature t over it (the samples of a tile sit in
 // shared memory, with their survival products so far); one CTA then adds the
-// CTAs' partials in CTA order and takes the argmin. ECE: 15 equal-width bins
-// of S per position, counts and sums per CTA in shared memory, then one pass
-// that adds the CTAs in order.
+// CTAs' partials in a fixed order and takes the argmin. ECE: 15 equal-width
+// bins of S per position, counts and sums per CTA in shared memory, then one
+// CTA per position that adds the CTAs in a fixed order.
 #include "calib.cuh"
 
 namespace dspark {
@@ -71,12 +71,21 @@ __global__ void __launch_bounds__(kCT) sts_nll_partials(CalibArgs a, int k) {
   a.partial[(long long)blockIdx.x * kCalGrid + t] = acc;
 }
 
-// Totals in CTA order, the argmin (lowest index on ties), T_k.
+// Totals over the CTAs (eight interleaved running sums per grid temperature,
+// added in a fixed order), the argmin (lowest index on ties), T_k.
 __global__ void __launch_bounds__(kCT) sts_argmin(CalibArgs a, int k) {
   __shared__ double s_loss[kCalGrid];
   const int t = threadIdx.x;
+  constexpr int kLanes = 8;
+  static_assert(kCalBlocks % kLanes == 0, "whole groups of CTAs");
+  double part[kLanes] = {};
+  for (int b = 0; b < kCalBlocks; b += kLanes) {
+#pragma unroll
+    for (int j = 0; j < kLanes; ++j) part[j] += a.partial[(long long)(b + j) * kCalGrid + t];
+  }
   double tot = 0.0;
-  for (int b = 0; b < kCalBlocks; ++b) tot += a.partial[(long long)b * kCalGrid + t];
+#pragma unroll
+  for (int j = 0; j < kLanes; ++j) tot += part[j];
   s_loss[t] = tot;
   __syncthreads();
   if (t == 0) {
@@ -113,23 +122,34 @@ __global__ void __launch_bounds__(kCT) ece_partials(CalibArgs a, int fitted) {
   for (int i = threadIdx.x; i < nb; i += kCT) out[i] = s_bins[i];
 }
 
-// ECE of every position from the CTAs' bins, added in CTA order.
-__global__ void __launch_bounds__(64) ece_finalize(CalibArgs a, float* ece) {
-  const int k = threadIdx.x;
-  if (k >= a.K) return;
+// ECE of position blockIdx.x from the CTAs' bins. Per bin, thread t adds the
+// CTAs t, t + kCT, ... in order, then a fixed tree adds the threads' sums.
+__global__ void __launch_bounds__(kCT) ece_finalize(CalibArgs a, float* ece) {
+  __shared__ double s_sum[3][kCT];
+  const int k = blockIdx.x, t = threadIdx.x;
   const int nb = a.K * kCalBins * 3;
   double e = 0.0;
   for (int bin = 0; bin < kCalBins; ++bin) {
-    double cnt = 0.0, sp = 0.0, sy = 0.0;
-    for (int b = 0; b < kCalBlocks; ++b) {
+    double v[3] = {0.0, 0.0, 0.0};
+    for (int b = t; b < kCalBlocks; b += kCT) {
       const double* c = a.bins + (long long)b * nb + (k * kCalBins + bin) * 3;
-      cnt += c[0];
-      sp += c[1];
-      sy += c[2];
+#pragma unroll
+      for (int f = 0; f < 3; ++f) v[f] += c[f];
     }
+#pragma unroll
+    for (int f = 0; f < 3; ++f) s_sum[f][t] = v[f];
+    __syncthreads();
+    for (int w = kCT / 2; w > 0; w >>= 1) {
+      if (t < w)
+#pragma unroll
+        for (int f = 0; f < 3; ++f) s_sum[f][t] += s_sum[f][t + w];
+      __syncthreads();
+    }
+    const double cnt = s_sum[0][0], sp = s_sum[1][0], sy = s_sum[2][0];
     if (cnt > 0.0) e += cnt / a.N * fabs(sp / cnt - sy / cnt);
+    __syncthreads();  // s_sum is refilled for the next bin
   }
-  ece[k] = (float)e;
+  if (t == 0) ece[k] = (float)e;
 }
 
 }  // namespace
@@ -153,7 +173,7 @@ cudaError_t calib_launch(CalibArgs a, void* ws, float* ece_before, float* ece_af
   }
   if (ece_before) {
     ece_partials<<<kCalBlocks, kCT, ece_smem, s>>>(a, 0);
-    ece_finalize<<<1, 64, 0, s>>>(a, ece_before);
+    ece_finalize<<<a.K, kCT, 0, s>>>(a, ece_before);
   }
   for (int k = 0; k < a.K; ++k) {
     sts_nll_partials<<<kCalBlocks, kCT, 0, s>>>(a, k);
@@ -161,7 +181,7 @@ cudaError_t calib_launch(CalibArgs a, void* ws, float* ece_before, float* ece_af
   }
   if (ece_after) {
     ece_partials<<<kCalBlocks, kCT, ece_smem, s>>>(a, 1);
-    ece_finalize<<<1, 64, 0, s>>>(a, ece_after);
+    ece_finalize<<<a.K, kCT, 0, s>>>(a, ece_after);
   }
   return cudaGetLastError();
 }

@@ -7,7 +7,10 @@ namespace dspark {
 
 constexpr int kCalGrid = 256;    // grid temperatures, log-spaced on [0.05, 20]
 constexpr int kCalBins = 15;     // equal-width ECE bins of S on [0, 1]
-constexpr int kCalBlocks = 256;  // CTAs of the sample-parallel passes
+// CTAs of the sample-parallel passes: one resident wave on B200 (6 CTAs of
+// 256 threads on each of 148 SMs), so that the fp64 exp / log chains of
+// enough warps overlap
+constexpr int kCalBlocks = 888;
 
 struct CalibArgs {
   const float* z;          // [N, K] confidence logits

@@ -46,8 +46,8 @@ def test_workspace_sizes(lib):
     assert bn.workspace_bytes(bn.OP_DRAFT, 4, 4, 1001, 16, bn.F32) == 0  # V % 8
     assert bn.workspace_bytes(bn.OP_VERIFY, 4, 65, 1024, 16, bn.F32) == 0  # K > 64
     assert bn.workspace_bytes(9, 4, 4, 1024, 16, bn.F32) == 0
-    # calibration: status block, 256 x 256 fp64 losses, 256 x K x 15 x 3 fp64 bin sums
-    assert bn.workspace_bytes(bn.OP_CALIB, 1000, 5, 0, 0, 0) == 256 + 256 * 256 * 8 + 256 * 5 * 15 * 3 * 8
+    # calibration: status block, 888 CTAs x 256 fp64 losses, 888 x K x 15 x 3 fp64 bin sums
+    assert bn.workspace_bytes(bn.OP_CALIB, 1000, 5, 0, 0, 0) == 256 + 888 * 256 * 8 + 888 * 5 * 15 * 3 * 8
     assert bn.workspace_bytes(bn.OP_CALIB, 1000, 65, 0, 0, 0) == 0
 
 
