@@ -262,3 +262,7 @@ def test_verify_with_and_without_the_draft_normalisers(cuda_ok):
             for k in range(w.K):
                 q = 2.0 ** (d[b, k, x[b, k]] * cs - qn[b, k, 0]) / qn[b, k, 1]
                 assert abs(q - rnd.q_tok[b, k].item()) <= 1e-5 * max(q, 1e-30)
+                # and the log normaliser: ln sum exp(d / temp) = (max + log2 sum) ln 2
+                lse = (qn[b, k, 0] + np.log2(qn[b, k, 1])) * np.log(2.0)
+                ql = rnd.q_lse[b, k].item()
+                assert abs(lse - ql) <= 1e-5 * max(1.0, abs(ql)), (b, k, lse, ql)
