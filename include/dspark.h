@@ -306,6 +306,23 @@ const char* dspark_status_string(int code);
 /* ABI version of this header: (major << 16) | minor. */
 int dspark_version(void);
 
+/*
+ * dspark_selftest_waits — makes the library's bounded device waits run out.
+ * One thread waits on an mbarrier phase that no arrival completes, then at a
+ * grid barrier that it reaches alone. Each wait gives up after the limit every
+ * kernel of the library uses (2 s of the GPU's global timer), reports
+ * DSPARK_STATUS_TIMEOUT in the status block (wait site 30) and lets the kernel
+ * return, so the context stays usable; the call takes about 4 s of GPU time.
+ * For tests of failure detection; nothing else calls it.
+ *   result    [2] i32 device, out: 1 where the mbarrier wait / the grid-barrier
+ *             wait gave up, 0 where it completed
+ *   ws        workspace of at least 256 bytes (its status block is used,
+ *             including the grid-barrier counter at byte 64)
+ * Errors: DSPARK_ERR_INVALID_ARG (null pointer, workspace too small or
+ * misaligned), DSPARK_ERR_UNSUPPORTED (no sm_100 device), DSPARK_ERR_CUDA.
+ */
+int dspark_selftest_waits(int32_t* result, void* ws, size_t ws_bytes, dspark_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,7 @@ SIGNATURES = {
     "dspark_clear_status": (_i, [_p, _p]),
     "dspark_status_string": (ctypes.c_char_p, [_i]),
     "dspark_version": (_i, []),
+    "dspark_selftest_waits": (_i, [_p, _p, _sz, _p]),
 }
 
 
@@ -259,6 +260,16 @@ def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, s
     _on_gpu(dev)
     rc = lib().dspark_sts_fit(*args, _stream(stream))
     _check(rc, "dspark_sts_fit")
+
+
+def selftest_waits(result, ws, stream=None) -> None:
+    """dspark_selftest_waits: an mbarrier wait and a grid-barrier wait that must give
+    up after the kernels' 2 s limit; result [2] int32 gets 1 for each that gave up."""
+    dev = ws.device
+    args = (_ptr(result, "result", torch.int32, (2,), dev), _ptr(ws, "ws", None, None, dev),
+            ws.numel() * ws.element_size())
+    _on_gpu(dev)
+    _check(lib().dspark_selftest_waits(*args, _stream(stream)), "dspark_selftest_waits")
 
 
 def read_status(ws, stream=None) -> Tuple[int, int]:

@@ -10,11 +10,16 @@
 #include "schedule.cuh"
 #include "verify.cuh"
 
+namespace dspark {
+// defined in selftest.cu
+cudaError_t selftest_waits_launch(Status* st, int32_t* result, cudaStream_t s);
+}  // namespace dspark
+
 using namespace dspark;
 
 namespace {
 
-constexpr int kAbiVersion = (2 << 16) | 0;
+constexpr int kAbiVersion = (2 << 16) | 1;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -50,6 +55,14 @@ inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? DSPARK_OK : DS
 extern "C" {
 
 int dspark_version(void) { return kAbiVersion; }
+
+int dspark_selftest_waits(int32_t* result, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  if (!result || !ws || !aligned16(ws) || ws_bytes < kStatusBytes) return DSPARK_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int e = device_check(&sms)) return e;
+  return cuda_status(
+      selftest_waits_launch(static_cast<Status*>(ws), result, (cudaStream_t)stream));
+}
 
 const char* dspark_status_string(int code) {
   switch (code) {

@@ -49,6 +49,9 @@ int main(void) {
         DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_read_status(NULL, NULL, &code, &first) == DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_clear_status(NULL, NULL) == DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_selftest_waits(NULL, ws, sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_selftest_waits(i32, NULL, sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_selftest_waits(i32, ws, 64, NULL) == DSPARK_ERR_INVALID_ARG);
 
   if (fails)
     printf("c abi: %d failures\n", fails);
