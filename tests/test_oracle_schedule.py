@@ -113,3 +113,36 @@ def test_load_trims_budget():
         if prev is not None:
             assert L.sum() <= prev
         prev = L.sum()
+
+
+def test_cost_rule_is_optimal_for_non_decreasing_costs():
+    """Against brute force over every per-request prefix vector: when the step
+    costs never decrease (a convex C(n), as in every cost table here), the
+    early-stopping walk reaches the least cost per emitted token, max A/C, of
+    the latency equation ("DSpark turns speculation into a scheduler", "The
+    speculative loop"). Why it must: for a fixed count of admitted drafts the
+    largest S form per-request prefixes and maximise A, and adding a draft
+    moves A/C towards S/step (a mediant), which only falls along the walk, so
+    A/C rises and then only falls."""
+    import itertools
+    rng = np.random.default_rng(5)
+    for trial in range(300):
+        B, K = int(rng.integers(1, 4)), int(rng.integers(1, 4))
+        z = rng.normal(1.0, 2.0, (B, K))
+        _, S = o.survival(z, np.linspace(1.0, 1.6, K))
+        n = B * (K + 1)
+        if trial % 2:
+            cost = 0.2 + np.cumsum(rng.exponential(0.3, n))           # strictly rising
+        else:
+            at = int(rng.integers(B, n + 1))                           # one step, as DSpark-5
+            cost = np.where(np.arange(1, n + 1) <= at, 1.0, float(rng.uniform(1.0, 3.0)))
+        fixed = float(rng.uniform(0.0, 2.0 * B))
+        L, _ = o.prefix_cut(S, cost, fixed)
+
+        def ratio(Lv):
+            m = int(np.sum(Lv))
+            A = B + sum(S[b, :Lv[b]].sum() for b in range(B))
+            return A / (fixed + cost[:B + m].sum())
+
+        best = max(ratio(Lv) for Lv in itertools.product(range(K + 1), repeat=B))
+        assert ratio(L) >= best * (1.0 - 1e-12), (trial, L.tolist(), ratio(L), best)
