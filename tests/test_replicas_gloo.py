@@ -68,3 +68,37 @@ def test_two_gloo_ranks_independent_batches():
     for r, out in ((0, out0), (1, out1)):
         ref, _ = _round_for(replicas.rank_workload(base, r))
         assert np.array_equal(out, ref)
+
+
+def _worker_leaves(rank, world, port, q):
+    import time
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), WORLD_SIZE=str(world),
+                      RANK=str(rank), LOCAL_RANK=str(rank))
+    from speculative_decoding_draft_sample_b200 import replicas
+    replicas.init("gloo", timeout_s=5)
+    if rank == 1:          # leaves between steps, with nothing in flight
+        q.put((1, "left", 0.0))
+        return
+    t0 = time.monotonic()
+    try:
+        replicas.barrier()  # the next collective of the timing bookkeeping
+        q.put((0, "no error", time.monotonic() - t0))
+    except Exception as e:  # noqa: BLE001 - any error ends the wait; a hang would not
+        q.put((0, type(e).__name__, time.monotonic() - t0))
+
+
+def test_a_rank_that_leaves_is_detected_not_waited_for():
+    """A rank that exits between steps makes the other rank's next collective
+    fail within the process group's short timeout instead of hanging it."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_leaves, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict((r, (what, dt)) for r, what, dt in (q.get(timeout=120) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+    assert res[1][0] == "left"
+    what, dt = res[0]
+    assert what != "no error" and dt < 60.0, res
