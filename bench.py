@@ -148,61 +148,93 @@ def time_region(fn, stream, iters: int) -> float:
     return e0.elapsed_time(e1) / iters
 
 
-def cpu_baseline(w: wl.Workload, inp_small, n_req: int, round_id: int, mode: int = bn.CUT_COST,
-                 threshold: float = 0.0):
-    """The fp64 oracle on a bounded sample of the round (n_req requests)."""
-    from oracle import dspark as o
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
+ORACLE_SAMPLE = 64  # requests per oracle step (cpu_baseline and the reference arm)
+
+
+def oracle_sample_inputs(w: wl.Workload, small, n_req: int):
+    """fp64 oracle inputs for the first n_req requests of the round (the
+    schedule's inputs cover the whole batch: the cut is batch-wide)."""
     reqs = list(range(n_req))
     part = wl.generate(w, reqs)
     rid = np.asarray(reqs)
-    oi = dict(target=part["target"].double().numpy(), base=part["base"].double().numpy(),
-              U=inp_small["U"].double().numpy(), W=inp_small["W"].double().numpy(),
-              last_tok=np.asarray(inp_small["last_tok"])[rid],
-              bias_scale=np.asarray(inp_small["bias_scale"], np.float64)[rid],
-              temp=np.asarray(inp_small["temp"], np.float64)[rid],
-              conf_logit=np.asarray(inp_small["conf_logit"], np.float64),
-              pos_temp=np.asarray(inp_small["pos_temp"], np.float64),
-              step_cost=np.asarray(inp_small["step_cost"], np.float64),
-              fixed_cost=float(inp_small["fixed_cost"]), dtype=w.dtype, request_ids=rid)
+    return dict(target=part["target"].double().numpy(), base=part["base"].double().numpy(),
+                U=small["U"].double().numpy(), W=small["W"].double().numpy(),
+                last_tok=np.asarray(small["last_tok"])[rid],
+                bias_scale=np.asarray(small["bias_scale"], np.float64)[rid],
+                temp=np.asarray(small["temp"], np.float64)[rid],
+                conf_logit=np.asarray(small["conf_logit"], np.float64),
+                pos_temp=np.asarray(small["pos_temp"], np.float64),
+                step_cost=np.asarray(small["step_cost"], np.float64),
+                fixed_cost=float(small["fixed_cost"]), dtype=w.dtype, request_ids=rid)
+
+
+def host_cores():
+    """(logical cores of this host, BLAS threads numpy uses)."""
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        blas = 1
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count() or 1
+    return int(cores), int(blas)
+
+
+def oracle_step(o, oi, round_id: int, mode: int, threshold: float):
+    """One step of the oracle module ``o`` on prepared inputs: (seconds, accepted drafts)."""
     t0 = time.perf_counter()
     r = o.run_round(oi, wl.PHILOX_SEED, round_id, mode, threshold)
-    dt = time.perf_counter() - t0
-    rounds = n_req / w.B
-    return dict(value=rounds / dt, unit=UNIT, cores=int(cores), kind="oracle",
-                sample=f"{n_req} of {w.B} requests of one round (draft with the rank-{w.r} bias, "
-                       f"batch-wide cut, verify), fp64 numpy, scaled by {w.B}/{n_req}",
-                seconds=dt, accepted=int(r["verify"]["a"].sum()))
+    return time.perf_counter() - t0, int(r["verify"]["a"].sum())
+
+
+def sample_text(w: wl.Workload, n_req: int) -> str:
+    return (f"{n_req} of {w.B} requests of one round per step (draft with the rank-{w.r} bias, "
+            f"the batch-wide cut, verify), fp64 numpy; rounds/s = ({n_req}/{w.B}) / step seconds")
+
+
+def cpu_baseline(w: wl.Workload, small, n_req: int, round_id: int, mode: int = bn.CUT_COST,
+                 threshold: float = 0.0):
+    """The fp64 oracle on a bounded sample of the round (n_req requests)."""
+    from oracle import dspark as o
+    oi = oracle_sample_inputs(w, small, n_req)
+    dt, acc = oracle_step(o, oi, round_id, mode, threshold)
+    cores, blas = host_cores()
+    return dict(value=(n_req / w.B) / dt, unit=UNIT, cores=cores, blas_threads=blas, kind="oracle",
+                sample=sample_text(w, n_req), seconds=dt, accepted=acc)
 
 
 def reference_arm(args, w: wl.Workload):
-    world, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    """The oracle timed on the host cores: every step runs it on the same
+    ORACLE_SAMPLE-request sample of the round, so ms_per_step is the time one
+    step really took and steps x ms_per_step is the time spent."""
+    rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     small = wl.small_inputs(w)
-    n_req = 4
+    n_req = min(ORACLE_SAMPLE, w.B)
     mode = CUT_MODES[args.cut]
     threshold = args.threshold if mode == bn.CUT_THRESHOLD else 0.0
+    from oracle import dspark as o
+    oi = oracle_sample_inputs(w, small, n_req)
     for i in range(args.warmup):
-        cpu_baseline(w, small, 1, 1000 + i, mode, threshold)
-    secs = 0.0
-    last = None
+        oracle_step(o, oi, 0, mode, threshold)
+    t0 = time.perf_counter()
     for i in range(args.steps):
-        last = cpu_baseline(w, small, n_req, i, mode, threshold)
-        secs += last["seconds"]
+        oracle_step(o, oi, 0, mode, threshold)
+    secs = time.perf_counter() - t0
     value = args.steps * (n_req / w.B) / secs
+    cores, blas = host_cores()
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": 1000.0 / value, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
-                       "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else "")},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
-                             "sample": last["sample"]},
+                       "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else ""),
+                       "step": f"{n_req} of {w.B} requests"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "blas_threads": blas,
+                             "kind": "oracle", "sample": sample_text(w, n_req)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -438,8 +470,9 @@ def main():
     }
     if (rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name
             and mode == bn.CUT_COST):
-        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), 128, 0).items()
-                                if k in ("value", "unit", "cores", "kind", "sample")}
+        line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), ORACLE_SAMPLE,
+                                                              0).items()
+                                if k in ("value", "unit", "cores", "blas_threads", "kind", "sample")}
     del graph  # released before the process group goes away
     replicas.finish()
     if rank == 0:

@@ -348,6 +348,101 @@ def prefix_cut(S: np.ndarray, step_cost: np.ndarray, fixed_cost: float,
     return L, flag
 
 
+def cut_alternatives(S: np.ndarray, step_cost: np.ndarray, fixed_cost: float,
+                     mode: int = 0, threshold: float = 0.0):
+    """The other cuts a flagged near-tie of ``prefix_cut`` leaves possible.
+
+    A device that evaluates the same rule in a different rounding order may
+    decide a near-tied comparison the other way, but only that comparison:
+    every other decision of the walk follows from it. So each alternative
+    flips exactly one flagged decision and walks on by the rule:
+
+    * mode 0, an admission test within CUT_WINDOW of its boundary at walk
+      position i: if the test admitted, the walk stops at i instead; if it
+      was the stopping test, the draft is admitted and the walk goes on.
+    * mode 0, survival products within CUT_WINDOW of each other on both
+      sides of the stopping point (a device may order them the other way):
+      the admitted draft and the first refused one trade places.
+    * mode 1, a survival product within CUT_WINDOW of the threshold: that
+      request's count moves by one.
+
+    Returns a list of cut vectors [B] (empty when nothing was flagged). A
+    check that adopts a device's cut only when it equals one of these still
+    catches any cut that differs elsewhere.
+    """
+    S = np.asarray(S, np.float64)
+    B, K = S.shape
+    alts = []
+    if mode == 2:
+        return alts
+    if mode == 1:
+        L = (S >= threshold).sum(axis=1).astype(np.int64)
+        near = np.abs(S - threshold) <= CUT_WINDOW * max(abs(threshold), 1e-300)
+        for b, k in zip(*np.nonzero(near)):
+            alt = L.copy()
+            alt[b] = k if S[b, k] >= threshold else k + 1
+            alts.append(alt)
+        return alts
+    cost = np.asarray(step_cost, np.float64)
+    items = sorted(((S[b, k], k, b) for b in range(B) for k in range(K)),
+                   key=lambda t: (-t[0], t[1], t[2]))
+    n = len(items)
+
+    def walk(order, flip):
+        """Admitted count per request; the decision at walk position ``flip``
+        (0-based, or -1 for none) is inverted. Also returns the stop and the
+        near-tied positions seen."""
+        A = float(B)
+        C = float(fixed_cost) + cost[:B].sum()
+        L = np.zeros(B, np.int64)
+        near = []
+        stop = n
+        for i, (s, k, b) in enumerate(order):
+            c = cost[B + i]
+            lhs, rhs = s * C, A * c
+            if abs(lhs - rhs) <= CUT_WINDOW * max(abs(lhs), abs(rhs)):
+                near.append(i)
+            admit = lhs >= rhs
+            if i == flip:
+                admit = not admit
+            if not admit:
+                stop = i
+                break
+            A += s
+            C += c
+            L[b] += 1
+        return L, stop, near
+
+    L0, stop, near = walk(items, -1)
+    for i in near:
+        alts.append(walk(items, i)[0])
+    if 0 < stop < n:
+        # near-equal survival products straddling the stopping point
+        s_in = items[stop - 1][0]
+        s_out = items[stop][0]
+        lo = [i for i in range(stop) if items[i][0] - s_out <= CUT_WINDOW * items[i][0]]
+        hi = [i for i in range(stop, n) if s_in - items[i][0] <= CUT_WINDOW * s_in]
+        for i in lo:
+            for j in hi:
+                order = list(items)
+                order[i], order[j] = order[j], order[i]
+                alts.append(walk(order, -1)[0])
+    return [a for a in alts if not np.array_equal(a, L0)]
+
+
+def adopt_cut(L: np.ndarray, alts, L_device: np.ndarray):
+    """The cut parity compares against: the oracle's own ``L``, or the
+    device's cut when it equals one of the flagged alternatives ``alts``.
+    Returns (cut, requests changed by adopting it)."""
+    L_device = np.asarray(L_device, np.int64)
+    if np.array_equal(L, L_device):
+        return L, 0
+    for alt in alts:
+        if np.array_equal(alt, L_device):
+            return L_device.copy(), int((L_device != L).sum())
+    return L, 0
+
+
 # --------------------------------------------------------------------------
 # a5, a6, a7: lossless verification, residual / bonus, emitted tokens
 # --------------------------------------------------------------------------
@@ -491,12 +586,15 @@ def run_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
     c, S = survival(inp["conf_logit"], inp["pos_temp"])
     L, cut_flag = prefix_cut(S, inp["step_cost"], inp["fixed_cost"], mode, threshold)
     forced = dr["forced"]
+    cut_forced = 0
     if cut_flag and teacher is not None:
-        tl = np.asarray(teacher["L"], np.int64)
-        forced += int((tl != L).sum())
-        L = tl
+        # only a cut that one flagged decision explains is adopted
+        alts = cut_alternatives(S, inp["step_cost"], inp["fixed_cost"], mode, threshold)
+        L, cut_forced = adopt_cut(L, alts, teacher["L"])
+        forced += cut_forced
     rid = inp.get("request_ids")
     Lr = L if rid is None else L[np.asarray(rid, np.int64)]
     vr = verify(inp["target"], dr["d"], dr["x"], Lr, inp["temp"], seed, round_id, rid, teacher)
     forced += vr["forced"]
-    return dict(draft=dr, c=c, S=S, L=L, cut_flag=cut_flag, verify=vr, forced=forced)
+    return dict(draft=dr, c=c, S=S, L=L, cut_flag=cut_flag, cut_forced=cut_forced, verify=vr,
+                forced=forced)

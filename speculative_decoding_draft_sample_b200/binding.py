@@ -119,10 +119,26 @@ def _on_gpu(device: torch.device) -> None:
         raise DSparkError(f"the call's tensors must be CUDA tensors, not on {device}")
 
 
-def _stream(stream) -> Optional[int]:
+def _stream(stream, device: torch.device) -> int:
+    """The handle of `stream`, or of `device`'s current stream; a stream of
+    another device is refused (its kernels would run there with this
+    device's pointers)."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        return torch.cuda.current_stream(device).cuda_stream
+    if stream.device != device:
+        raise DSparkError(f"the stream is on {stream.device}, the call's tensors on {device}")
     return stream.cuda_stream
+
+
+def _call(name: str, device: torch.device, args, stream) -> None:
+    """Calls entry point `name` with `device` current: the library launches
+    on the current device and looks up per-device state there, so it must be
+    the device that holds the call's tensors."""
+    _on_gpu(device)
+    s = _stream(stream, device)
+    with torch.cuda.device(device):
+        rc = getattr(lib(), name)(*args, s)
+    _check(rc, name)
 
 
 def workspace_bytes(op: int, B: int, K: int, V: int, r: int, dtype: int) -> int:
@@ -150,9 +166,7 @@ def draft_sample(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: in
         _ptr(q_lse, "q_lse", f32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
         _ptr(q_norm, "q_norm", f32, (B, K, 2), dev), _ptr(ws, "ws", None, None, dev),
         ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_draft_sample(*args, _stream(stream))
-    _check(rc, "dspark_draft_sample")
+    _call("dspark_draft_sample", dev, args, stream)
 
 
 def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, stream=None) -> None:
@@ -169,9 +183,7 @@ def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, strea
         _ptr(temp, "temp", f32, (B,), dev), B, K, V, r, dt, int(k),
         _ptr(d, "d", base.dtype, (B, K, V), dev), _ptr(ws, "ws", None, None, dev),
         ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_draft_logits(*args, _stream(stream))
-    _check(rc, "dspark_draft_logits")
+    _call("dspark_draft_logits", dev, args, stream)
 
 
 def draft_pick(d, last_tok, temp, seed: int, round_id: int, k: int, x, q_lse, q_tok, ws,
@@ -185,9 +197,7 @@ def draft_pick(d, last_tok, temp, seed: int, round_id: int, k: int, x, q_lse, q_
         _ptr(x, "x", i32, (B, K), dev), _ptr(q_lse, "q_lse", f32, (B, K), dev),
         _ptr(q_tok, "q_tok", f32, (B, K), dev), _ptr(q_norm, "q_norm", f32, (B, K, 2), dev),
         _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_draft_pick(*args, _stream(stream))
-    _check(rc, "dspark_draft_pick")
+    _call("dspark_draft_pick", dev, args, stream)
 
 
 def draft_sample_static(base, U, W, bias_scale, last_tok, temp, seed: int, round_id: int,
@@ -206,9 +216,7 @@ def draft_sample_static(base, U, W, bias_scale, last_tok, temp, seed: int, round
         _ptr(x, "x", i32, (B, K), dev), _ptr(d, "d", base.dtype, (B, K, V), dev),
         _ptr(q_lse, "q_lse", f32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
         _ptr(status_out, "status_out", i32, (2,), dev))
-    _on_gpu(dev)
-    rc = lib().dspark_draft_sample_static(*args, _stream(stream))
-    _check(rc, "dspark_draft_sample_static")
+    _call("dspark_draft_sample_static", dev, args, stream)
 
 
 def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: int,
@@ -222,9 +230,7 @@ def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: in
         float(threshold), _ptr(cut, "cut", torch.int32, (B,), dev),
         _ptr(survival, "survival", f32, (B, K), dev), _ptr(ws, "ws", None, None, dev),
         ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_prefix_schedule(*args, _stream(stream))
-    _check(rc, "dspark_prefix_schedule")
+    _call("dspark_prefix_schedule", dev, args, stream)
 
 
 def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out, n_emit,
@@ -242,9 +248,7 @@ def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, o
         _ptr(accepted, "accepted", i32, (B,), dev), _ptr(out, "out", i32, (B, K1), dev),
         _ptr(n_emit, "n_emit", i32, (B,), dev), _ptr(ws, "ws", None, None, dev),
         ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_verify(*args, _stream(stream))
-    _check(rc, "dspark_verify")
+    _call("dspark_verify", dev, args, stream)
 
 
 def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, stream=None) -> None:
@@ -257,9 +261,7 @@ def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, s
         _ptr(T_out, "T_out", f32, (K,), dev), _ptr(index_out, "index_out", torch.int32, (K,), dev),
         _ptr(ece_before, "ece_before", f32, (K,), dev), _ptr(ece_after, "ece_after", f32, (K,), dev),
         _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    rc = lib().dspark_sts_fit(*args, _stream(stream))
-    _check(rc, "dspark_sts_fit")
+    _call("dspark_sts_fit", dev, args, stream)
 
 
 def selftest_waits(result, ws, stream=None) -> None:
@@ -268,19 +270,25 @@ def selftest_waits(result, ws, stream=None) -> None:
     dev = ws.device
     args = (_ptr(result, "result", torch.int32, (2,), dev), _ptr(ws, "ws", None, None, dev),
             ws.numel() * ws.element_size())
-    _on_gpu(dev)
-    _check(lib().dspark_selftest_waits(*args, _stream(stream)), "dspark_selftest_waits")
+    _call("dspark_selftest_waits", dev, args, stream)
 
 
 def read_status(ws, stream=None) -> Tuple[int, int]:
     """(status bits, first offending request or -1); synchronises and clears."""
     code = ctypes.c_uint32(0)
     first = ctypes.c_int32(-1)
-    rc = lib().dspark_read_status(_ptr(ws, "ws"), _stream(stream), ctypes.byref(code),
-                                  ctypes.byref(first))
+    p = _ptr(ws, "ws")
+    dev = ws.device
+    s = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        rc = lib().dspark_read_status(p, s, ctypes.byref(code), ctypes.byref(first))
     _check(rc, "dspark_read_status")
     return int(code.value), int(first.value)
 
 
 def clear_status(ws, stream=None) -> None:
-    _check(lib().dspark_clear_status(_ptr(ws, "ws"), _stream(stream)), "dspark_clear_status")
+    p = _ptr(ws, "ws")
+    dev = ws.device
+    s = _stream(stream, dev)
+    with torch.cuda.device(dev):
+        _check(lib().dspark_clear_status(p, s), "dspark_clear_status")

@@ -50,7 +50,7 @@ class SpecRound:
         for both. The two calls share the workspace: they only meet in its
         status block, which both update atomically.
         """
-        main = stream if stream is not None else torch.cuda.current_stream()
+        main = stream if stream is not None else torch.cuda.current_stream(self.x.device)
 
         def schedule(s):
             bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
@@ -58,6 +58,8 @@ class SpecRound:
                                self.ws, s)
 
         if side_stream is not None:
+            if side_stream.device != self.x.device or main.device != self.x.device:
+                raise bn.DSparkError(f"the round's streams must be on {self.x.device}")
             fork, join = torch.cuda.Event(), torch.cuda.Event()
             fork.record(main)
             side_stream.wait_event(fork)

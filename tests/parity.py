@@ -87,7 +87,9 @@ def check_round(w: wl.Workload, inp: Dict[str, object], rnd: SpecRound, requests
     assert np.array_equal(dr["x"], g["x"]), "drafted tokens differ"
     np.testing.assert_allclose(g["q_tok"], dr["q_tok"], rtol=RTOL)
     np.testing.assert_allclose(g["q_lse"], dr["q_lse"], rtol=RTOL, atol=1e-6)
-    # schedule
+    # schedule: the whole batch's cut. At a flagged near-tie the oracle adopts
+    # the GPU's cut only if one flipped decision explains it (cut_alternatives),
+    # so every request the flip does not touch is still compared with the oracle
     np.testing.assert_allclose(g["S"], r["S"], rtol=RTOL)
     assert np.array_equal(r["L"], g["L"]), "prefix cuts differ"
     # verify + emit
@@ -95,6 +97,7 @@ def check_round(w: wl.Workload, inp: Dict[str, object], rnd: SpecRound, requests
     assert np.array_equal(vr["a"], g["a"]), "accepted lengths differ"
     assert np.array_equal(vr["out"], g["out"]), "emitted tokens differ"
     assert np.array_equal(vr["n_emit"], g["n_emit"])
-    return dict(forced=int(r["forced"]), d_flags=int(dr["d_flag"].sum()),
+    return dict(forced=int(r["forced"]), cut_flag=bool(r["cut_flag"]),
+                cut_forced=int(r["cut_forced"]), d_flags=int(dr["d_flag"].sum()),
                 x_flags=int(dr["x_flag"].sum()), acc_flags=int(vr["acc_flag"].sum()),
                 y_flags=int(vr["y_flag"].sum()), accepted=int(g["a"].sum()))

@@ -48,20 +48,41 @@ def test_cut_modes(cuda_ok, mode, threshold):
         assert np.all(L == 0) and np.all(rnd.n_emit.cpu().numpy() == 1)
 
 
-FULL = [wl.DSPARK5, wl.QWEN3, wl.sweep(4), wl.sweep(16), wl.STRESS]
+FULL = [wl.DSPARK5, wl.QWEN3, wl.sweep(4), wl.sweep(8), wl.sweep(12), wl.sweep(16), wl.STRESS]
+
+
+def sampled_requests(w, inp, rnd, n=32, seed=0):
+    """At least ``n`` requests of a full-size round: the first and last row of
+    every 128-request M-tile of the draft kernel (0, 127, 128, 255, ..., B-1),
+    one request of every (cut, accepted) class the round produced, the special
+    request kinds of the stress mix, then random ones."""
+    rng = np.random.default_rng(seed)
+    reqs = {0, w.B - 1}
+    for m0 in range(0, w.B, 128):
+        reqs |= {m0, min(m0 + 127, w.B - 1)}
+    cut = rnd.cut.cpu().numpy()
+    acc = rnd.accepted.cpu().numpy()
+    for c, a in sorted(set(zip(cut.tolist(), acc.tolist()))):
+        reqs.add(int(rng.choice(np.nonzero((cut == c) & (acc == a))[0])))
+    for kind in ("identical", "independent"):
+        if np.any(inp[kind]):
+            reqs.add(int(np.nonzero(inp[kind])[0][0]))
+    greedy = np.nonzero(np.asarray(inp["temp"]) == 0)[0]
+    if len(greedy):
+        reqs.add(int(greedy[0]))
+    rest = [b for b in rng.permutation(w.B).tolist() if b not in reqs]
+    reqs |= set(rest[:max(0, n - len(reqs))])
+    return sorted(reqs)
 
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
 def test_full_size_sampled_requests(cuda_ok, w):
-    rng = np.random.default_rng(0)
     inp = wl.generate(w)
     rnd, _ = run_gpu(w, inp, 0)
-    reqs = sorted(set([0, w.B - 1] + list(rng.choice(w.B, size=4, replace=False))))
-    if w is wl.STRESS:  # make sure the special request kinds are covered
-        reqs = sorted(set(reqs + [int(np.nonzero(inp["identical"])[0][0]),
-                                  int(np.nonzero(inp["independent"])[0][0]),
-                                  int(np.nonzero(np.asarray(inp["temp"]) == 0)[0][0])]))
-    check_round(w, inp, rnd, reqs, 0)
+    reqs = sampled_requests(w, inp, rnd)
+    assert len(reqs) >= min(32, w.B)
+    stats = check_round(w, inp, rnd, reqs, 0)
+    print(w.name, len(reqs), "requests", stats)
 
 
 def test_lossless_on_gpu(cuda_ok):

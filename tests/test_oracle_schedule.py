@@ -146,3 +146,120 @@ def test_cost_rule_is_optimal_for_non_decreasing_costs():
 
         best = max(ratio(Lv) for Lv in itertools.product(range(K + 1), repeat=B))
         assert ratio(L) >= best * (1.0 - 1e-12), (trial, L.tolist(), ratio(L), best)
+
+
+def _order(S):
+    B, K = S.shape
+    return sorted(((S[b, k], k, b) for b in range(B) for k in range(K)),
+                  key=lambda t: (-t[0], t[1], t[2]))
+
+
+def _walk_state(S, cost, fixed, upto):
+    """(A, C) of the early-stopping walk before walk position ``upto`` (0-based),
+    assuming every earlier draft was admitted."""
+    B = S.shape[0]
+    A, C = float(B), fixed + cost[:B].sum()
+    for i, (s, _, _) in enumerate(_order(S)[:upto]):
+        A += s
+        C += cost[B + i]
+    return A, C
+
+
+def _off_by_one_cut(S, cost, fixed):
+    """The cost rule with its per-draft step cost read one slot late: a plausible
+    indexing slip of a device kernel, written here to check that parity sees it."""
+    B = S.shape[0]
+    A, C = float(B), fixed + cost[:B].sum()
+    L = np.zeros(B, np.int64)
+    for j, (s, k, b) in enumerate(_order(S), start=1):
+        c = cost[min(B + j, len(cost) - 1)]     # should be cost[B + j - 1]
+        if s * C >= A * c:
+            A, C = A + s, C + c
+            L[b] += 1
+        else:
+            break
+    return L
+
+
+def _flagged_case(rng):
+    """A random cut whose walk holds an exact tie at an early admitted draft: its
+    step cost is set so that S_i C_i = A_i c_i, which flags the cut."""
+    B, K = int(rng.integers(4, 12)), int(rng.integers(2, 6))
+    z = rng.normal(1.0, 1.5, (B, K))
+    _, S = o.survival(z, np.linspace(1.0, 1.6, K))
+    n = B * (K + 1)
+    at = int(rng.integers(B + 2, n))
+    cost = np.where(np.arange(1, n + 1) <= at, 1.0, float(rng.uniform(1.2, 2.5)))
+    fixed = float(B)
+    L, _ = o.prefix_cut(S, cost, fixed)
+    stop = int(L.sum())
+    if stop < 4:
+        return None
+    i = int(rng.integers(0, stop - 3))
+    A, C = _walk_state(S, cost, fixed, i)
+    cost = cost.copy()
+    cost[B + i] = _order(S)[i][0] * C / A
+    return S, cost, fixed, i
+
+
+def test_cut_alternatives_flip_one_decision():
+    """Every alternative of a flagged cut is the walk with one near-tied decision
+    inverted; the device's cut is adopted only when it is one of them."""
+    rng = np.random.default_rng(11)
+    seen = 0
+    for trial in range(400):
+        case = _flagged_case(rng)
+        if case is None:
+            continue
+        S, cost, fixed, i = case
+        L, flag = o.prefix_cut(S, cost, fixed)
+        assert flag
+        alts = o.cut_alternatives(S, cost, fixed)
+        assert alts, "a flagged cut has at least one alternative"
+        order = _order(S)
+        stop_at_i = np.zeros(S.shape[0], np.int64)
+        for s, k, b in order[:i]:
+            stop_at_i[b] += 1
+        # the tie at draft i: either the walk stops there, or the oracle stopped
+        # there and the alternative admits it
+        assert any(np.array_equal(a, stop_at_i) for a in alts) or np.array_equal(L, stop_at_i)
+        cut, changed = o.adopt_cut(L, alts, alts[0])
+        assert np.array_equal(cut, alts[0]) and changed == int((alts[0] != L).sum())
+        seen += 1
+    assert seen >= 100
+
+
+def test_cut_parity_catches_off_by_one_despite_a_flag():
+    """A device cut with an off-by-one in the step-cost index is refused even
+    when a near-tie elsewhere in the walk flags the round: only a cut that one
+    flagged decision explains is adopted, never the device's whole vector."""
+    rng = np.random.default_rng(12)
+    refused = adopted = 0
+    for trial in range(600):
+        case = _flagged_case(rng)
+        if case is None:
+            continue
+        S, cost, fixed, _ = case
+        L, flag = o.prefix_cut(S, cost, fixed)
+        bad = _off_by_one_cut(S, cost, fixed)
+        if not flag or np.array_equal(bad, L):
+            continue
+        alts = o.cut_alternatives(S, cost, fixed)
+        cut, changed = o.adopt_cut(L, alts, bad)
+        if np.array_equal(cut, L) and changed == 0:
+            refused += 1
+        else:
+            adopted += 1
+    assert refused >= 50, (refused, adopted)
+    # the slip coincides with a legitimate flip only by chance
+    assert adopted <= 0.1 * (refused + adopted), (refused, adopted)
+
+
+def test_threshold_cut_alternatives():
+    S = np.array([[0.9, 0.5 * (1 + 1e-9), 0.1], [0.8, 0.7, 0.6]])
+    L, flag = o.prefix_cut(S, None, 0.0, mode=1, threshold=0.5)
+    assert flag and L.tolist() == [2, 3]
+    alts = o.cut_alternatives(S, None, 0.0, mode=1, threshold=0.5)
+    assert [a.tolist() for a in alts] == [[1, 3]]
+    assert o.adopt_cut(L, alts, np.array([2, 2]))[0].tolist() == [2, 3]   # not a flagged flip
+    assert o.adopt_cut(L, alts, np.array([1, 3]))[0].tolist() == [1, 3]
