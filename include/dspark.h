@@ -11,6 +11,8 @@
  *   dspark_sts_fit         Sequential Temperature Scaling of the confidences, ECE
  *   dspark_verify          lossless rejection-sampling verification, residual or
  *                          bonus token, accepted lengths and emitted tokens
+ *                          (dspark_verify_target_stats / dspark_verify_from_stats:
+ *                          its two halves, so the first can run beside the draft)
  *
  * Sources, cited by page title and section:
  *   [P1] "DSpark turns speculation into a scheduler" (benebsworth.pages.dev)
@@ -82,8 +84,10 @@ enum { DSPARK_CUT_COST = 0, DSPARK_CUT_THRESHOLD = 1, DSPARK_CUT_NONE = 2 };
 /*
  * Workspace bytes needed by operation `op` (DSPARK_OP_*) for these sizes
  * (r is ignored except by DSPARK_OP_DRAFT). Pure host function. Returns 0 for
- * unsupported arguments. One workspace of the largest size may serve all three
- * operations on one stream.
+ * unsupported arguments. One workspace of the largest size may serve all the
+ * operations of a round: the draft's chunk partials and verification's target
+ * statistics occupy different regions of it, so dspark_verify_target_stats may
+ * run beside dspark_draft_sample; otherwise the calls must not overlap.
  */
 size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype);
 
@@ -183,8 +187,9 @@ int dspark_draft_pick(const void* d, const int32_t* last_tok, const float* temp,
  *
  *   conf_logit [B, K] f32, pos_temp [K] f32 (> 0), step_cost [B*(K+1)] f32
  *   cut [B] i32 out, survival [B, K] f32 out
- * Limits: 1 <= K <= 64; the cost rule needs B*K <= 8192 (one CTA sorts all
- * drafts), the other modes take any B >= 1.
+ * Limits: 1 <= K <= 64; the cost rule needs B*K <= 16384 (one CTA sorts all
+ * drafts, so that the call fits beside the draft kernel on the SMs it leaves
+ * free), the other modes take any B >= 1.
  */
 int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp,
                            const float* step_cost, float fixed_cost, int B, int K,
@@ -209,7 +214,13 @@ int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp,
  * cut[b] (purpose 3, position a+1). Greedy requests (temp 0) accept iff
  * x == argmax of the target row and emit argmax of target row a.
  * out[b] = x[b,0..a-1], y, then -1 up to K+1 entries; n_emit[b] = a + 1.
- * Only target rows 0..a and draft row a are read.
+ *
+ * Two launches on `stream`: dspark_verify_target_stats (one streaming pass over
+ * target rows 0..cut[b] of every request, which leaves each row's softmax
+ * partials in the workspace), then dspark_verify_from_stats (the acceptance
+ * tests from those normalisers, one pass over target row a and draft row a of
+ * every rejected request for the residual, a one-chunk rescan for the bonus).
+ * Target rows past cut[b] and draft rows other than a are never read.
  *
  *   target [B, K+1, V] dtype, d [B, K, V] dtype, x [B, K] i32,
  *   q_tok [B, K] f32, cut [B] i32 or NULL (all K), temp [B] f32
@@ -227,6 +238,40 @@ int dspark_verify(const void* target, const void* d, const int32_t* x,
                   uint64_t round_id, int32_t* accepted, int32_t* out,
                   int32_t* n_emit, void* ws, size_t ws_bytes,
                   dspark_stream_t stream);
+
+/*
+ * The two halves of dspark_verify, for callers that start the first one as
+ * soon as the cut is known, beside the draft (it needs neither d, x nor the
+ * draft's probabilities). Calling dspark_verify_target_stats and then
+ * dspark_verify_from_stats with the same target, cut, temp and workspace gives
+ * results identical to dspark_verify (the same kernels run).
+ * [P1] intro and "Caveats"; [P2] "Sources"; [P3] "Speculative Decoding in Two
+ * Sentences".
+ *
+ * dspark_verify_target_stats: for every request b and target row j <= cut[b]
+ *   (all K + 1 rows when cut is NULL), the softmax partials of every 2 KB
+ *   chunk of the row, (max z, sum 2^(z - max z)) of z = target * log2(e) /
+ *   temp[b], or (max, lowest argmax) for temp[b] == 0, written to the
+ *   workspace's statistics region. The region lies past the draft's partials
+ *   of a workspace of the same size, so this call may run on another stream
+ *   concurrently with dspark_draft_sample on that workspace; it must complete
+ *   before dspark_verify_from_stats starts (an event or the same stream).
+ * dspark_verify_from_stats: everything else dspark_verify does, reading the
+ *   statistics instead of the target rows' normalisers. Its arguments are
+ *   dspark_verify's; cut and temp must be the ones the statistics were made
+ *   with.
+ * Both take a workspace of dspark_workspace_bytes(DSPARK_OP_VERIFY, ...) bytes.
+ */
+int dspark_verify_target_stats(const void* target, const int32_t* cut,
+                               const float* temp, int B, int K, int V, int dtype,
+                               void* ws, size_t ws_bytes, dspark_stream_t stream);
+
+int dspark_verify_from_stats(const void* target, const void* d, const int32_t* x,
+                             const float* q_tok, const float* q_norm,
+                             const int32_t* cut, const float* temp, int B, int K,
+                             int V, int dtype, uint64_t seed, uint64_t round_id,
+                             int32_t* accepted, int32_t* out, int32_t* n_emit,
+                             void* ws, size_t ws_bytes, dspark_stream_t stream);
 
 /*
  * Sequential Temperature Scaling of the per-position confidences, and their

@@ -28,10 +28,13 @@ def _softmax(z: np.ndarray) -> np.ndarray:
 
 
 def output_distribution(target: np.ndarray, base: np.ndarray, U: np.ndarray, W: np.ndarray,
-                        last_tok: int, scale: float, tau: float, L: int) -> Dict[Tuple[int, ...], float]:
+                        last_tok: int, scale: float, tau: float, L: int,
+                        R: np.ndarray = None) -> Dict[Tuple[int, ...], float]:
     """P(emitted tokens = seq) for every emitted sequence seq of one request.
 
     target [K+1, V], base [K, V], U [V, r], W [r, V]; all fp64, tau > 0.
+    With R [r, r] the bias comes from the recurrent state
+    h_k = U[x_{k-1}] + tanh(h_{k-1} @ R) (h_0 = 0) instead of U[x_{k-1}].
     """
     target = np.asarray(target, np.float64)
     base = np.asarray(base, np.float64)
@@ -40,27 +43,31 @@ def output_distribution(target: np.ndarray, base: np.ndarray, U: np.ndarray, W: 
     V = target.shape[1]
     dist: Dict[Tuple[int, ...], float] = defaultdict(float)
 
-    def walk(k: int, prev: int, prefix: Tuple[int, ...], weight: float) -> None:
-        # ``weight`` = P(drafts x_1..x_{k-1} == prefix and all of them accepted)
+    r = U.shape[1]
+
+    def walk(k: int, prev: int, prefix: Tuple[int, ...], weight: float, h: np.ndarray) -> None:
+        # ``weight`` = P(drafts x_1..x_{k-1} == prefix and all of them accepted);
+        # h: the recurrent state of position k - 1
         if k > L:
             p = _softmax(target[L] / tau)
             for yv in range(V):
                 dist[prefix + (yv,)] += weight * p[yv]
             return
-        q = _softmax((base[k - 1] + scale * (U[prev] @ W)) / tau)
+        hk = U[prev] if R is None else U[prev] + np.tanh(h @ R)
+        q = _softmax((base[k - 1] + scale * (hk @ W)) / tau)
         p = _softmax(target[k - 1] / tau)
         resid = np.maximum(0.0, p - q)
-        R = resid.sum()
+        rsum = resid.sum()
         for xv in range(V):
             if q[xv] == 0.0:
                 continue
             alpha = min(1.0, p[xv] / q[xv])
-            walk(k + 1, xv, prefix + (xv,), weight * q[xv] * alpha)
-            if alpha < 1.0 and R > 0:
+            walk(k + 1, xv, prefix + (xv,), weight * q[xv] * alpha, hk)
+            if alpha < 1.0 and rsum > 0:
                 w_rej = weight * q[xv] * (1.0 - alpha)
                 for yv in range(V):
                     if resid[yv] > 0:
-                        dist[prefix + (yv,)] += w_rej * resid[yv] / R
+                        dist[prefix + (yv,)] += w_rej * resid[yv] / rsum
 
-    walk(1, int(last_tok), (), 1.0)
+    walk(1, int(last_tok), (), 1.0, np.zeros(r))
     return dict(dist)

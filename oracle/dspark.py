@@ -36,6 +36,11 @@ Readings where the pages are silent (each marked R<n> below):
 * R6  the early-stopping prefix cut (see ``prefix_cut``).
 * R7  acceptance is strict: accept iff u < p(x)/q(x).
 * R8  a residual of exact zero (floating point only) falls back to p.
+* R11 the recurrent head (the pages name an optional head that tracks the
+      whole block prefix and give no equations): a state h_k in R^r,
+      h_0 = 0, h_k = U[x_{k-1}] + tanh(h_{k-1} @ R), stored in the logits'
+      dtype, and bias_k = scale_b * h_k @ W. With R = 0 it is the Markov head
+      bit for bit.
 * Greedy requests (temperature 0) draft argmax d, accept iff the draft
   equals argmax of the target row, and emit argmax of the target row;
   ties go to the lowest index.
@@ -137,6 +142,41 @@ def draft_logits(base_k: np.ndarray, bias: np.ndarray, dtype: str,
     return out, flag
 
 
+def recurrent_state(U: np.ndarray, R: np.ndarray, prev: np.ndarray, h_prev: np.ndarray,
+                    dtype: str):
+    """The recurrent head's state for one position (R11), every request.
+
+    h = round_storage(U[prev] + tanh(h_prev @ R)) with h_prev [B, r] the
+    previous position's stored state (zeros before the first position), so
+    that the state carries the whole drafted prefix, not only the previous
+    token ([P1] "DSpark's semi-autoregressive compromise": recurrent head
+    machinery beside the Markov head; [P3] "The Semi-Autoregressive Trick": an
+    optional head that tracks the full block prefix).
+
+    Returns (h [B, r], flag [B, r]). For bf16 storage an element is flagged
+    when its fp64 value lies within the error of a device computing it in fp32
+    of a rounding midpoint: the fp32 accumulation of r products (r 2^-23
+    sum_j |h_j R_ji|), tanh to 2^-22 relative, and the final fp32 add
+    (2^-22 |v|).
+    """
+    U = np.asarray(U, np.float64)
+    R = np.asarray(R, np.float64)
+    h_prev = np.asarray(h_prev, np.float64)
+    a = h_prev @ R
+    th = np.tanh(a)
+    v = U[np.asarray(prev, np.int64)] + th
+    if dtype != "bf16":
+        return round_to_storage(v, dtype)
+    r = R.shape[0]
+    m, e = np.frexp(v)
+    sc = m * 256.0
+    out = np.ldexp(np.rint(sc), e - 8)
+    mid = np.ldexp(np.trunc(sc) + np.sign(sc) * 0.5, e - 8)
+    win = 2.0 ** -22 * (np.abs(v) + np.abs(th)) + r * 2.0 ** -23 * (np.abs(h_prev) @ np.abs(R))
+    flag = np.isfinite(v) & (np.abs(v - mid) <= win)
+    return out, flag
+
+
 def inverse_cdf(w: np.ndarray, u: np.ndarray, window: float = U_WINDOW, normalized: bool = True):
     """Inverse-CDF draw from unnormalised non-negative weights, per row (R4).
 
@@ -201,13 +241,21 @@ def sample_position(d: np.ndarray, tau: np.ndarray, u: np.ndarray) -> Dict[str, 
     return dict(x=x, q_lse=q_lse, q_tok=q_tok, flag=flag)
 
 
-def draft_position(base_k, U, W, prev, scale, tau, u, dtype: str) -> Dict[str, np.ndarray]:
-    """One draft position for every request: bias, stored d, and the draw."""
+def draft_position(base_k, U, W, prev, scale, tau, u, dtype: str,
+                   h: Optional[np.ndarray] = None) -> Dict[str, np.ndarray]:
+    """One draft position for every request: bias, stored d, and the draw.
+
+    The bias multiplies W by U[prev] (Markov head) or, when given, by the
+    recurrent state h [B, r] (R11)."""
     Uf = np.asarray(U, np.float64)
     Wf = np.asarray(W, np.float64)
-    bias = markov_bias(Uf, Wf, prev, scale)
-    babs = np.abs(np.asarray(scale, np.float64))[:, None] * (
-        np.abs(Uf[np.asarray(prev, np.int64)]) @ np.abs(Wf))
+    if h is None:
+        bias = markov_bias(Uf, Wf, prev, scale)
+        rows = Uf[np.asarray(prev, np.int64)]
+    else:
+        rows = np.asarray(h, np.float64)
+        bias = np.asarray(scale, np.float64)[:, None] * (rows @ Wf)
+    babs = np.abs(np.asarray(scale, np.float64))[:, None] * (np.abs(rows) @ np.abs(Wf))
     d, d_flag = draft_logits(base_k, bias, dtype, babs, Uf.shape[1])
     s = sample_position(d, tau, u)
     return dict(d=d, d_flag=d_flag, x=s["x"], q_lse=s["q_lse"], q_tok=s["q_tok"],
@@ -219,11 +267,14 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
     """All K positions of the semi-autoregressive draft (a1 + a2).
 
     For k = 1..K: bias from x_{k-1} (x_0 = last committed token, R2), the
-    stored draft logits d_k, then x_k ~ softmax(d_k / tau).
+    stored draft logits d_k, then x_k ~ softmax(d_k / tau). With ``inp["R"]``
+    [r, r] the bias comes from the recurrent state h_k of R11 instead of
+    U[x_{k-1}] alone; the states are returned as ``h`` [B, K, r].
 
-    Teacher forcing: with ``teacher`` (the GPU's "d" [B,K,V] and "x" [B,K]),
-    a flagged d element takes the teacher's value and a flagged draw takes
-    the teacher's token; ``forced`` counts how often that changed anything.
+    Teacher forcing: with ``teacher`` (the GPU's "d" [B,K,V] and "x" [B,K],
+    and "h" [B,K,r] for the recurrent head), a flagged d or h element takes
+    the teacher's value and a flagged draw takes the teacher's token;
+    ``forced`` counts how often that changed anything.
     """
     base = inp["base"]
     B, K, V = base.shape
@@ -237,10 +288,24 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
     d_flag = np.zeros((B, K), bool)
     x_flag = np.zeros((B, K), bool)
     forced = 0
+    Rm = inp.get("R")
+    r = np.shape(inp["U"])[1]
+    hs = np.zeros((B, K, r)) if Rm is not None else None
+    h_flag = np.zeros((B, K), bool)
+    h = np.zeros((B, r))
     for k in range(1, K + 1):
         u = uniform(seed, req, k, PURPOSE_DRAFT, round_id)
+        if Rm is not None:
+            h, hf = recurrent_state(inp["U"], Rm, prev, h, inp["dtype"])
+            if teacher is not None and hf.any():
+                th = np.asarray(teacher["h"][:, k - 1], np.float64)
+                diff = hf & (th != h)
+                forced += int(diff.sum())
+                h = np.where(hf, th, h)
+            hs[:, k - 1] = h
+            h_flag[:, k - 1] = hf.any(axis=1)
         st = draft_position(base[:, k - 1], inp["U"], inp["W"], prev, inp["bias_scale"],
-                            tau, u, inp["dtype"])
+                            tau, u, inp["dtype"], h if Rm is not None else None)
         if teacher is not None and st["d_flag"].any():
             td = np.asarray(teacher["d"][:, k - 1], np.float64)
             diff = st["d_flag"] & (td != st["d"])
@@ -267,7 +332,7 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
         x_flag[:, k - 1] = st["x_flag"]
         prev = st["x"]
     return dict(d=d, d_flag=d_flag, x=x, q_lse=q_lse, q_tok=q_tok, x_flag=x_flag,
-                forced=forced)
+                h=hs, h_flag=h_flag, forced=forced)
 
 
 # --------------------------------------------------------------------------

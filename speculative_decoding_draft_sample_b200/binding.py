@@ -38,6 +38,9 @@ SIGNATURES = {
     "dspark_prefix_schedule": (_i, [_p, _p, _p, _f, _i, _i, _i, _f, _p, _p, _p, _sz, _p]),
     "dspark_verify": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p, _p, _p,
                            _p, _sz, _p]),
+    "dspark_verify_target_stats": (_i, [_p, _p, _p, _i, _i, _i, _i, _p, _sz, _p]),
+    "dspark_verify_from_stats": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _u64, _u64, _p,
+                                      _p, _p, _p, _sz, _p]),
     "dspark_draft_logits": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p,
                                  _sz, _p]),
     "dspark_draft_pick": (_i, [_p, _p, _p, _i, _i, _i, _i, _u64, _u64, _i, _p, _p, _p, _p, _p,
@@ -233,9 +236,8 @@ def prefix_schedule(conf_logit, pos_temp, step_cost, fixed_cost: float, mode: in
     _call("dspark_prefix_schedule", dev, args, stream)
 
 
-def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out, n_emit,
-           ws, stream=None, q_norm=None) -> None:
-    """dspark_verify: target [B,K+1,V], d [B,K,V], x, q_tok [B,K], cut [B] -> accepted, out, n_emit."""
+def _verify_args(target, d, x, q_tok, cut, temp, seed, round_id, accepted, out, n_emit, ws,
+                 q_norm):
     B, K1, V = target.shape
     K = K1 - 1
     dt = _dtype_code(target)
@@ -248,7 +250,34 @@ def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, o
         _ptr(accepted, "accepted", i32, (B,), dev), _ptr(out, "out", i32, (B, K1), dev),
         _ptr(n_emit, "n_emit", i32, (B,), dev), _ptr(ws, "ws", None, None, dev),
         ws.numel() * ws.element_size())
+    return dev, args
+
+
+def verify(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out, n_emit,
+           ws, stream=None, q_norm=None) -> None:
+    """dspark_verify: target [B,K+1,V], d [B,K,V], x, q_tok [B,K], cut [B] -> accepted, out, n_emit."""
+    dev, args = _verify_args(target, d, x, q_tok, cut, temp, seed, round_id, accepted, out, n_emit,
+                             ws, q_norm)
     _call("dspark_verify", dev, args, stream)
+
+
+def verify_target_stats(target, cut, temp, ws, stream=None) -> None:
+    """dspark_verify_target_stats: softmax partials of target rows 0..cut[b] into ws."""
+    B, K1, V = target.shape
+    dev = target.device
+    args = (_ptr(target, "target", None, (B, K1, V), dev),
+            _ptr(cut, "cut", torch.int32, (B,), dev), _ptr(temp, "temp", torch.float32, (B,), dev),
+            B, K1 - 1, V, _dtype_code(target), _ptr(ws, "ws", None, None, dev),
+            ws.numel() * ws.element_size())
+    _call("dspark_verify_target_stats", dev, args, stream)
+
+
+def verify_from_stats(target, d, x, q_tok, cut, temp, seed: int, round_id: int, accepted, out,
+                      n_emit, ws, stream=None, q_norm=None) -> None:
+    """dspark_verify_from_stats: dspark_verify after dspark_verify_target_stats."""
+    dev, args = _verify_args(target, d, x, q_tok, cut, temp, seed, round_id, accepted, out, n_emit,
+                             ws, q_norm)
+    _call("dspark_verify_from_stats", dev, args, stream)
 
 
 def sts_fit(conf_logit, survived, T_out, index_out, ece_before, ece_after, ws, stream=None) -> None:

@@ -19,13 +19,27 @@ using namespace dspark;
 
 namespace {
 
-constexpr int kAbiVersion = (2 << 16) | 1;
+constexpr int kAbiVersion = (3 << 16) | 0;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline int nchunks(int V) { return (V + kChunk - 1) / kChunk; }
+
+// Workspace layout shared by the calls of one round:
+//   [status block 256][draft chunk partials][target-row statistics][work counter 256]
+// The statistics sit past the draft's partials, so that dspark_verify_target_stats
+// may run on another stream while dspark_draft_sample runs (they share only the
+// status block, which both update atomically).
+inline size_t draft_region(int B, int V) { return round_up((size_t)B * nchunks(V) * sizeof(float2), 256); }
+inline size_t stats_region(int B, int K, int V, int dtype) {
+  return round_up((size_t)B * (K + 1) * stats_chunks(V, dtype) * sizeof(float2), 256);
+}
+inline size_t stats_offset(int B, int V) { return kStatusBytes + draft_region(B, V); }
+inline size_t counter_offset(int B, int K, int V, int dtype) {
+  return stats_offset(B, V) + stats_region(B, K, V, dtype);
+}
 
 bool shape_ok(int B, int K, int V, int dtype) {
   if (dtype != DSPARK_F32 && dtype != DSPARK_BF16) return false;
@@ -80,7 +94,7 @@ size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype) {
   switch (op) {
     case DSPARK_OP_DRAFT:
       if (!shape_ok(B, K, V, dtype) || r < 1 || r > 1024) return 0;
-      return kStatusBytes + round_up((size_t)B * nchunks(V) * sizeof(float2), 256);
+      return kStatusBytes + draft_region(B, V);
     case DSPARK_OP_SCHEDULE:
       if (B < 1 || K < 1 || K > 64) return 0;
       return kStatusBytes;
@@ -89,7 +103,7 @@ size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype) {
       return calib_workspace_bytes(B, K);
     case DSPARK_OP_VERIFY:
       if (!shape_ok(B, K, V, dtype)) return 0;
-      return kStatusBytes;
+      return counter_offset(B, K, V, dtype) + 256;
     default:
       return 0;
   }
@@ -221,7 +235,8 @@ int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp, const
     return DSPARK_ERR_INVALID_ARG;
   if (mode == DSPARK_CUT_COST && !step_cost) return DSPARK_ERR_INVALID_ARG;
   if (B < 1 || K < 1 || K > 64) return DSPARK_ERR_INVALID_ARG;
-  if (mode == DSPARK_CUT_COST && (long long)B * K > kMaxScheduleItems) return DSPARK_ERR_UNSUPPORTED;
+  if (mode == DSPARK_CUT_COST && ((long long)B * K > kMaxScheduleItems || B > kMaxScheduleItems))
+    return DSPARK_ERR_UNSUPPORTED;
   if (!aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
   if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_SCHEDULE, B, K, 8, 1, DSPARK_F32))
     return DSPARK_ERR_WORKSPACE;
@@ -241,19 +256,46 @@ int dspark_prefix_schedule(const float* conf_logit, const float* pos_temp, const
   return cuda_status(prefix_schedule_launch(a, (cudaStream_t)stream));
 }
 
-int dspark_verify(const void* target, const void* d, const int32_t* x, const float* q_tok,
-                  const float* q_norm,
-                  const int32_t* cut, const float* temp, int B, int K, int V, int dtype,
-                  uint64_t seed, uint64_t round_id, int32_t* accepted, int32_t* out,
-                  int32_t* n_emit, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int stats_prepare(StatsArgs& sa, int* sms, const void* target, const int32_t* cut, const float* temp,
+                  int B, int K, int V, int dtype, void* ws, size_t ws_bytes) {
+  if (!target || !temp || !ws) return DSPARK_ERR_INVALID_ARG;
+  if (!shape_ok(B, K, V, dtype)) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(target) || !aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
+  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_VERIFY, B, K, V, 1, dtype)) return DSPARK_ERR_WORKSPACE;
+  if (int e = device_check(sms)) return e;
+  char* w = static_cast<char*>(ws);
+  sa.target = target;
+  sa.cut = cut;
+  sa.temp = temp;
+  sa.B = B;
+  sa.K = K;
+  sa.V = V;
+  sa.dtype = dtype;
+  sa.partials = reinterpret_cast<float2*>(w + stats_offset(B, V));
+  sa.nchunk = stats_chunks(V, dtype);
+  sa.next = reinterpret_cast<unsigned long long*>(w + counter_offset(B, K, V, dtype));
+  sa.status = static_cast<Status*>(ws);
+  return DSPARK_OK;
+}
+
+int verify_decide(const void* target, const void* d, const int32_t* x, const float* q_tok,
+                  const float* q_norm, const int32_t* cut, const float* temp, int B, int K, int V,
+                  int dtype, uint64_t seed, uint64_t round_id, int32_t* accepted, int32_t* out,
+                  int32_t* n_emit, void* ws, size_t ws_bytes, cudaStream_t s, bool with_stats) {
   if (!target || !d || !x || !q_tok || !temp || !accepted || !out || !n_emit || !ws)
     return DSPARK_ERR_INVALID_ARG;
-  if (!shape_ok(B, K, V, dtype)) return DSPARK_ERR_INVALID_ARG;
-  if (!aligned16(target) || !aligned16(d) || !aligned16(ws)) return DSPARK_ERR_INVALID_ARG;
-  if (ws_bytes < dspark_workspace_bytes(DSPARK_OP_VERIFY, B, K, V, 1, dtype))
-    return DSPARK_ERR_WORKSPACE;
+  if (!aligned16(d)) return DSPARK_ERR_INVALID_ARG;
+  StatsArgs sa;
   int sms = 0;
-  if (int e = device_check(&sms)) return e;
+  if (int e = stats_prepare(sa, &sms, target, cut, temp, B, K, V, dtype, ws, ws_bytes)) return e;
+  if (with_stats) {
+    cudaError_t e = target_stats_launch(sa, sms, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
   VerifyArgs a;
   a.target = target;
   a.d = d;
@@ -272,8 +314,41 @@ int dspark_verify(const void* target, const void* d, const int32_t* x, const flo
   a.out = out;
   a.n_emit = n_emit;
   a.status = static_cast<Status*>(ws);
+  a.stats = sa.partials;
+  a.nstat = sa.nchunk;
   const int C = verify_cluster_size(B, V, dtype, sms);
-  return cuda_status(verify_launch(a, C, (cudaStream_t)stream));
+  return cuda_status(verify_launch(a, C, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int dspark_verify_target_stats(const void* target, const int32_t* cut, const float* temp, int B,
+                               int K, int V, int dtype, void* ws, size_t ws_bytes,
+                               dspark_stream_t stream) {
+  StatsArgs sa;
+  int sms = 0;
+  if (int e = stats_prepare(sa, &sms, target, cut, temp, B, K, V, dtype, ws, ws_bytes)) return e;
+  return cuda_status(target_stats_launch(sa, sms, (cudaStream_t)stream));
+}
+
+int dspark_verify_from_stats(const void* target, const void* d, const int32_t* x,
+                             const float* q_tok, const float* q_norm, const int32_t* cut,
+                             const float* temp, int B, int K, int V, int dtype, uint64_t seed,
+                             uint64_t round_id, int32_t* accepted, int32_t* out, int32_t* n_emit,
+                             void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  return verify_decide(target, d, x, q_tok, q_norm, cut, temp, B, K, V, dtype, seed, round_id,
+                       accepted, out, n_emit, ws, ws_bytes, (cudaStream_t)stream, false);
+}
+
+int dspark_verify(const void* target, const void* d, const int32_t* x, const float* q_tok,
+                  const float* q_norm,
+                  const int32_t* cut, const float* temp, int B, int K, int V, int dtype,
+                  uint64_t seed, uint64_t round_id, int32_t* accepted, int32_t* out,
+                  int32_t* n_emit, void* ws, size_t ws_bytes, dspark_stream_t stream) {
+  return verify_decide(target, d, x, q_tok, q_norm, cut, temp, B, K, V, dtype, seed, round_id,
+                       accepted, out, n_emit, ws, ws_bytes, (cudaStream_t)stream, true);
 }
 
 int dspark_sts_fit(const float* conf_logit, const uint8_t* survived, int N, int K, float* T_out,

@@ -27,6 +27,8 @@ enum WaitSite : unsigned int {
   kWhereTcAccFull = 14,
   kWhereTcAccEmpty = 15,
   kWhereTcGrid = 16,
+  kWhereStatsEmpty = 20,
+  kWhereStatsFull = 21,
 };
 
 __device__ __forceinline__ void report_wait(Status* st, unsigned int site, int request) {

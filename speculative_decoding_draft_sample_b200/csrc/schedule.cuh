@@ -5,8 +5,9 @@
 
 namespace dspark {
 
-// Largest B*K one schedule call handles (one CTA, items sorted in shared memory).
-constexpr int kMaxScheduleItems = 8192;
+// Largest B*K the cost rule handles (one CTA, 8-byte keys sorted in shared memory).
+constexpr int kMaxScheduleItems = 16384;
+constexpr int kSchedThreads = 1024;
 
 struct SchedArgs {
   const float* conf_logit;  // [B, K]

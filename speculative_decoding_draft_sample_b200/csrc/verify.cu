@@ -325,25 +325,151 @@ struct VerifyCta {
     return block_online(m, sum);
   }
 
-  // Per-thread (max, lowest argmax) of the raw values and a NaN / +inf check.
-  __device__ void row_argmax(const T* row, float& mv, int& mi, float& chk) {
-    mv = -INFINITY;
-    mi = 0x7fffffff;
-    chk = -INFINITY;
-    pass(row, nullptr, 1, [&](int s, const unsigned char* a, const unsigned char*) {
-#pragma unroll
-      for (int q = 0; q < kVecs; ++q) {
-        const int e0 = vec_elem(s, q);
-        if (e0 >= n) continue;
-        float v[N];
-        Vec16<DT>::load(vec_ptr(a, q), v);
-#pragma unroll
-        for (int j = 0; j < N; ++j) {
-          chk = max_nan(chk, v[j]);
-          argmax_merge(mv, mi, v[j], lo + e0 + j);
-        }
+  // A target row's normaliser (max z, sum 2^(z - max z)) from its chunk
+  // partials, combined in the same order in every CTA.
+  __device__ float2 stats_norm(const float2* P, int nst) {
+    float m = -INFINITY, sum = 0.f;
+    for (int c = tid; c < nst; c += kVThreads) {
+      const float2 q = P[c];
+      online_merge(m, sum, q.x, q.y);
+    }
+    return block_online(m, sum);
+  }
+
+  // A greedy row's (max, lowest argmax) from its chunk partials; bad when a
+  // chunk reported NaN or +inf (its maximum is NaN).
+  __device__ void stats_argmax(const float2* P, int nst, float& mv, int& mi, bool& bad) {
+    float m = -INFINITY;
+    int i = 0x7fffffff;
+    bool b = false;
+    for (int c = tid; c < nst; c += kVThreads) {
+      const float2 q = P[c];
+      b |= (q.x != q.x);
+      argmax_merge(m, i, q.x, __float_as_int(q.y));
+    }
+    warp_argmax(m, i);
+    b = __any_sync(0xffffffffu, b);
+    if (lane == 0) {
+      red[warp] = m;
+      reinterpret_cast<int*>(red)[8 + warp] = i;
+      reinterpret_cast<int*>(red)[16 + warp] = b;
+    }
+    __syncthreads();
+    mv = red[0];
+    mi = reinterpret_cast<int*>(red)[8];
+    bad = reinterpret_cast<int*>(red)[16] != 0;
+    for (int w = 1; w < kVWarps; ++w) {
+      argmax_merge(mv, mi, red[w], reinterpret_cast<int*>(red)[8 + w]);
+      bad |= reinterpret_cast<int*>(red)[16 + w] != 0;
+    }
+    __syncthreads();
+  }
+
+  // Inclusive scan of one value per thread over the CTA (thread order); also
+  // returns the CTA total. Uses red[0..kVWarps).
+  __device__ float block_scan(float v, float& total) {
+    const float incl = warp_inclusive_scan(v);
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    float before = 0.f, tot = 0.f;
+    for (int w = 0; w < kVWarps; ++w) {
+      if (w < warp) before += red[w];
+      tot += red[w];
+    }
+    __syncthreads();
+    total = tot;
+    return before + incl;
+  }
+
+  // Inverse-CDF draw from the weights 2^(t cs - M) of a whole target row
+  // (index order, strict ">"; past the end: the last positive entry), with
+  // thr = u * Z. The crossing chunk is located from the row's chunk partials
+  // P (their masses rescaled to M), then only that chunk of the row is read
+  // again. Runs in one CTA; returns the token in every thread, -2 when no
+  // entry has positive weight.
+  __device__ int place_row(const T* row, const float2* P, int nst, int V, float thr, float cs, float M) {
+    int* found = sint;  // [0] crossing chunk, [1] last positive chunk
+    if (tid == 0) {
+      found[0] = 0x7fffffff;
+      found[1] = -1;
+    }
+    __syncthreads();
+    float before = 0.f;  // mass of the chunks of earlier rounds
+    float rem = -1.f;
+    for (int c0 = 0; c0 < nst; c0 += kVThreads) {
+      const int c = c0 + tid;
+      float w = 0.f;
+      if (c < nst) {
+        const float2 q = P[c];
+        w = (q.x == -INFINITY) ? 0.f : q.y * ex2(q.x - M);
       }
-    });
+      float tot;
+      const float incl = block_scan(w, tot);
+      if (w > 0.f) {
+        atomicMax(&found[1], c);
+        if (thr < before + incl) atomicMin(&found[0], c);
+      }
+      __syncthreads();
+      if (found[0] != 0x7fffffff) {
+        // this thread's exclusive prefix is read by the owner below
+        if (c == found[0]) red[16] = thr - (before + incl - w);
+        __syncthreads();
+        rem = red[16];
+        break;
+      }
+      before += tot;
+    }
+    int ch = found[0];
+    if (ch == 0x7fffffff) {  // rounding: past the total, the last positive chunk
+      ch = found[1];
+      rem = INFINITY;
+    }
+    __syncthreads();
+    if (ch < 0) return -2;
+    // rescan chunk ch: thread t weighs 16 bytes (N entries) in index order
+    constexpr int CE = kStatChunkBytes / E::kBytes;
+    const int e0 = ch * CE + tid * N;
+    float w[N];
+    float ts = 0.f;
+    const bool ok = e0 < V;
+    float v[N];
+    if (ok) Vec16<DT>::load(row + e0, v);
+#pragma unroll
+    for (int j = 0; j < N; ++j) {
+      w[j] = ok ? ex2(fmaf(v[j], cs, -M)) : 0.f;
+      ts += w[j];
+    }
+    float tot;
+    const float incl = block_scan(ts, tot);
+    if (tid == 0) {
+      sint[2] = 0x7fffffff;
+      sint[3] = -1;
+    }
+    __syncthreads();
+    if (ts > 0.f) {
+      atomicMax(&sint[3], tid);
+      if (rem < incl) atomicMin(&sint[2], tid);
+    }
+    __syncthreads();
+    int tt = sint[2];
+    const bool fallback = tt == 0x7fffffff;
+    if (fallback) tt = sint[3];
+    int tok = -2;
+    if (tid == tt) {
+      float r2 = rem - (incl - ts);
+      int f = -1, lp = -1;
+#pragma unroll
+      for (int j = 0; j < N; ++j) {
+        if (w[j] > 0.f) lp = j;
+        if (f < 0 && !fallback && w[j] > 0.f && r2 < w[j]) f = j;
+        if (f < 0) r2 -= w[j];
+      }
+      red[17] = __int_as_float(e0 + (f < 0 ? lp : f));
+    }
+    __syncthreads();
+    if (tt >= 0) tok = __float_as_int(red[17]);
+    __syncthreads();
+    return tok;
   }
 
   // Inverse-CDF placement of `thr` on the weights wfun(t_value, d_value) of
@@ -588,40 +714,21 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   bool badrow = false;
   float M = 0.f, Z = 0.f;  // current target row's max (z units) and sum
   int y = -1;
+  const float2* stat_b = a.stats + (long long)b * (K + 1) * a.nstat;
 
+  // The walk needs no pass over the rows: their normalisers come from the
+  // target statistics, and every CTA of the cluster takes the same decisions
+  // from the same partials.
   for (int j = 0; j <= L; ++j) {
     const T* row = target + (long long)j * V;
+    const float2* P = stat_b + (long long)j * a.nstat;
     const int xk = (j < L) ? a.x[(long long)b * K + j] : -1;
     if (j < L && (xk < 0 || xk >= V) && tid == 0 && c.rank == 0) report(st, DSPARK_STATUS_BAD_TOKEN, b);
     if (greedy) {
-      float mv, chk;
-      int mi;
-      c.row_argmax(row + c.lo, mv, mi, chk);
-      warp_argmax(mv, mi);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) chk = max_nan(chk, __shfl_xor_sync(0xffffffffu, chk, o));
-      if (c.lane == 0) {
-        red[c.warp] = mv;
-        red[8 + c.warp] = chk;
-        reinterpret_cast<int*>(red)[16 + c.warp] = mi;
-      }
-      __syncthreads();
-      float m = red[0], ck = red[8];
-      int mm = reinterpret_cast<int*>(red)[16];
-      for (int w = 1; w < kVThreads / 32; ++w) {
-        argmax_merge(m, mm, red[w], reinterpret_cast<int*>(red)[16 + w]);
-        ck = max_nan(ck, red[8 + w]);
-      }
-      __syncthreads();
-      const bool bad = (ck != ck) || ck == INFINITY;
-      c.gather(Exch{m, 0.f, 0.f, mm | (bad ? (int)0x80000000 : 0)});
-      float gm = -INFINITY;
-      int gi = 0x7fffffff;
-      bool gbad = false;
-      for (int r = 0; r < c.C; ++r) {
-        argmax_merge(gm, gi, got[r].f0, got[r].i0 & 0x7fffffff);
-        gbad |= got[r].i0 < 0;
-      }
+      float gm;
+      int gi;
+      bool gbad;
+      c.stats_argmax(P, a.nstat, gm, gi, gbad);
       if (gbad || gm == -INFINITY) {
         badrow = true;
         gi = 0;
@@ -634,36 +741,24 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
       ++acc;
       continue;
     }
-
-    // one online pass: (max, sum) of z = t * cs; t[x] of the draft being tested
-    // comes from the CTA whose slice holds x
-    const float2 mz = c.row_stats(row + c.lo, cs);
-    float tx = -INFINITY;
-    if (tid == 0 && xk >= c.lo && xk < c.lo + c.n) tx = E::load(row, xk) * cs;
-    c.gather(Exch{mz.x, mz.y, tx, 0});
-    float gtx = -INFINITY;
-    for (int r = 0; r < c.C; ++r) gtx = fmaxf(gtx, got[r].f2);
-    const float2 MZ = combine_ranks(got, c.C);
+    const float2 MZ = c.stats_norm(P, a.nstat);
     M = MZ.x;
     Z = MZ.y;
-    // rank totals rescaled to the row maximum, for a placement on this row
-    // (a separate array: every thread is still reading `got` above)
-    if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
-    __syncthreads();
     if (!(Z > 0.f) || Z == INFINITY || M == -INFINITY || M == INFINITY) {
       badrow = true;
       rejected = (j < L);
       y = 0;
       break;
     }
-    if (j == L) {  // every verified draft accepted: bonus token from p of row L
-      const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kBonus);
-      y = c.place(u * Z, rw, row + c.lo, nullptr,
-                  [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); },
-                  [&](float2 r) { return r.x == -INFINITY ? 0.f : r.y * ex2(r.x - M); });
+    if (j == L) {  // every verified draft accepted: bonus token from p of row L (rank 0 draws it)
+      if (c.rank == 0) {
+        const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kBonus);
+        y = c.place_row(row, P, a.nstat, V, u * Z, cs, M);
+      }
       break;
     }
-    const float p = ex2(gtx - M) / Z;
+    const float tx = (xk >= 0 && xk < V) ? E::load(row, xk) * cs : -INFINITY;
+    const float p = ex2(tx - M) / Z;
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(j + 1), kAccept);
     if (!(u < p / a.q_tok[(long long)b * K + j])) {
       rejected = true;
@@ -673,8 +768,8 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
   }
 
   if (rejected && !greedy && !badrow) {
-    // residual norm(max(0, p - q)) over target row acc and draft row acc
-    // (q = softmax(d / temp), its normaliser recomputed here)
+    // residual norm(max(0, p - q)) over target row acc and draft row acc: the
+    // one streaming pass of the kernel
     const T* trow = target + (long long)acc * V + c.lo;
     const T* drow = drow0 + (long long)acc * V + c.lo;
     // the draft row's normaliser: from the draw that produced it when the
@@ -696,7 +791,7 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
     float sr = 0.f, rs = 0.f;
     c.pass(trow, drow, 2, [&](int s, const unsigned char* ta, const unsigned char* da) {
       constexpr int N = Vec16<DT>::N;
-      float acc[2] = {0.f, 0.f};
+      float acc2[2] = {0.f, 0.f};
 #pragma unroll
       for (int q = 0; q < kVecs; ++q) {
         if (c.vec_elem(s, q) >= c.n) continue;
@@ -704,10 +799,10 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
         Vec16<DT>::load(c.vec_ptr(ta, q), tv);
         Vec16<DT>::load(c.vec_ptr(da, q), dv);
 #pragma unroll
-        for (int j = 0; j < N; ++j) acc[j & 1] += resid(tv[j], dv[j]);
+        for (int jj = 0; jj < N; ++jj) acc2[jj & 1] += resid(tv[jj], dv[jj]);
       }
-      sr += acc[0] + acc[1];
-      rs += acc[0] + acc[1];
+      sr += acc2[0] + acc2[1];
+      rs += acc2[0] + acc2[1];
       if (c.record_end(s)) {
         const float t = warp_sum(rs);
         if (c.lane == 0) rec[(s / c.G) * kVWarps + c.warp] = make_float2(0.f, t);
@@ -723,14 +818,10 @@ __global__ void __launch_bounds__(kVThreads, kVBlocksPerSM) verify_kernel(Verify
     const float u = uniform24(a.seed, a.round_id, (uint32_t)b, (uint32_t)(acc + 1), kResidual);
     if (R > 0.f) {
       y = c.place(u * R, rw, trow, drow, resid, [](float2 r) { return r.y; });
-    } else {
+    } else if (c.rank == 0) {
       // exact-zero residual (floating point only): draw from p instead
-      const float2 mz = c.row_stats(trow, cs);
-      c.gather(Exch{mz.x, mz.y, 0.f, 0});
-      if (tid < c.C) rw[tid] = (got[tid].f0 == -INFINITY) ? 0.f : got[tid].f1 * ex2(got[tid].f0 - M);
-      __syncthreads();
-      y = c.place(u * Z, rw, trow, nullptr, [&](float tv, float) { return ex2(fmaf(tv, cs, -M)); },
-                  [&](float2 r) { return r.x == -INFINITY ? 0.f : r.y * ex2(r.x - M); });
+      y = c.place_row(target + (long long)acc * V, stat_b + (long long)acc * a.nstat, a.nstat, V,
+                      u * Z, cs, M);
     }
   }
 

@@ -5,6 +5,26 @@
 
 namespace dspark {
 
+// Bytes of a target row per softmax partial of the row statistics
+// (1024 bf16 or 512 fp32 entries).
+constexpr int kStatChunkBytes = 2048;
+
+// Statistics of the target rows 0..cut[b] of every request (target_stats.cu).
+struct StatsArgs {
+  const void* target;        // [B, K+1, V]
+  const int32_t* cut;        // [B] or null (every request verifies K)
+  const float* temp;         // [B]
+  int B, K, V, dtype;
+  float2* partials;          // [B, K+1, nchunk] chunk partials (rows past the cut untouched)
+  int nchunk;                // stats_chunks(V, dtype)
+  unsigned long long* next;  // work counter, zeroed by the launcher
+  Status* status;
+};
+
+// 2 KB chunks per target row.
+int stats_chunks(int V, int dtype);
+cudaError_t target_stats_launch(const StatsArgs& a, int num_sms, cudaStream_t s);
+
 struct VerifyArgs {
   const void* target;     // [B, K+1, V]
   const void* d;          // [B, K, V]
@@ -20,6 +40,8 @@ struct VerifyArgs {
   int32_t* n_emit;        // [B]
   Status* status;
   int slice;              // vocabulary entries per CTA (multiple of 8)
+  const float2* stats;    // [B, K+1, nstat] target-row partials from target_stats
+  int nstat;              // stats_chunks(V, dtype)
 };
 
 // CTAs per request (the cluster size) for this batch shape.

@@ -34,7 +34,7 @@ class SpecRound:
         self.out = torch.empty((B, K + 1), **i32)
         self.n_emit = torch.empty((B,), **i32)
         nbytes = max(bn.workspace_bytes(op, B, K, V, r, code)
-                     for op in (bn.OP_DRAFT, bn.OP_SCHEDULE, bn.OP_VERIFY))
+                     for op in (bn.OP_DRAFT, bn.OP_SCHEDULE, bn.OP_VERIFY))  # verify's holds the draft's
         if nbytes == 0:
             raise bn.DSparkError(f"unsupported round shape B={B} K={K} V={V} r={r}")
         self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
@@ -44,18 +44,21 @@ class SpecRound:
             side_stream=None) -> None:
         """Issues the round on ``stream`` (no host synchronisation).
 
-        The prefix schedule needs only the confidence logits, so with a
-        ``side_stream`` it runs there, concurrently with the draft (the
-        one-launch draft kernel leaves SMs free for it); verification waits
-        for both. The two calls share the workspace: they only meet in its
-        status block, which both update atomically.
+        The prefix schedule needs only the confidence logits, and the target
+        rows' statistics only the target logits and the cut, so with a
+        ``side_stream`` both run there, concurrently with the draft (the
+        one-launch draft kernel leaves SMs free for them); the rest of
+        verification waits for both. The calls share the workspace: the draft's
+        partials and the statistics occupy different regions of it, and they
+        meet only in its status block, which every call updates atomically.
         """
         main = stream if stream is not None else torch.cuda.current_stream(self.x.device)
 
-        def schedule(s):
+        def schedule_and_stats(s):
             bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
                                float(inp["fixed_cost"]), mode, threshold, self.cut, self.survival,
                                self.ws, s)
+            bn.verify_target_stats(inp["target"], self.cut, inp["temp"], self.ws, s)
 
         if side_stream is not None:
             if side_stream.device != self.x.device or main.device != self.x.device:
@@ -63,17 +66,18 @@ class SpecRound:
             fork, join = torch.cuda.Event(), torch.cuda.Event()
             fork.record(main)
             side_stream.wait_event(fork)
-            schedule(side_stream)
+            schedule_and_stats(side_stream)
             join.record(side_stream)
         bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
                         inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
                         self.ws, main, q_norm=self.q_norm)
         if side_stream is None:
-            schedule(main)
+            schedule_and_stats(main)
         else:
             main.wait_event(join)
-        bn.verify(inp["target"], self.d, self.x, self.q_tok, self.cut, inp["temp"], seed,
-                  round_id, self.accepted, self.out, self.n_emit, self.ws, main, q_norm=self.q_norm)
+        bn.verify_from_stats(inp["target"], self.d, self.x, self.q_tok, self.cut, inp["temp"],
+                             seed, round_id, self.accepted, self.out, self.n_emit, self.ws, main,
+                             q_norm=self.q_norm)
 
     def status(self, stream=None):
         return bn.read_status(self.ws, stream)

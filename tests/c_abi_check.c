@@ -22,11 +22,13 @@ int main(void) {
   uint32_t code = 0;
   int32_t first = 0;
 
-  CHECK((dspark_version() >> 16) == 2);
+  CHECK((dspark_version() >> 16) == 3);
   /* draft: status block + one (max, sum) pair per request and 256-entry chunk */
   CHECK(dspark_workspace_bytes(DSPARK_OP_DRAFT, 256, 5, 129280, 256, DSPARK_BF16) ==
         256 + (size_t)256 * 505 * 8);
-  CHECK(dspark_workspace_bytes(DSPARK_OP_VERIFY, 256, 5, 129280, 256, DSPARK_BF16) == 256);
+  /* verify: status block, the draft's partials, per-chunk target-row statistics, a counter */
+  CHECK(dspark_workspace_bytes(DSPARK_OP_VERIFY, 256, 5, 129280, 256, DSPARK_BF16) ==
+        256 + (size_t)256 * 505 * 8 + (size_t)256 * 6 * 127 * 8 + 256);
   CHECK(dspark_workspace_bytes(DSPARK_OP_SCHEDULE, 1024, 8, 0, 0, 0) == 256);
   CHECK(dspark_workspace_bytes(DSPARK_OP_DRAFT, 4, 4, 1001, 16, DSPARK_F32) == 0); /* V % 8 */
   CHECK(dspark_workspace_bytes(DSPARK_OP_VERIFY, 4, 65, 1024, 16, DSPARK_F32) == 0); /* K > 64 */
@@ -45,6 +47,10 @@ int main(void) {
                                sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_verify(NULL, NULL, i32, f32, NULL, NULL, f32, 4, 4, 1024, DSPARK_F32, 1, 0, i32,
                       i32, i32, ws, sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_verify_target_stats(NULL, NULL, f32, 4, 4, 1024, DSPARK_F32, ws, sizeof ws, NULL) ==
+        DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_verify_from_stats(NULL, NULL, i32, f32, NULL, NULL, f32, 4, 4, 1024, DSPARK_F32, 1,
+                                 0, i32, i32, i32, ws, sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_sts_fit(NULL, NULL, 10, 5, f32, NULL, NULL, NULL, ws, sizeof ws, NULL) ==
         DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_read_status(NULL, NULL, &code, &first) == DSPARK_ERR_INVALID_ARG);

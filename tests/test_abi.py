@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_strings(lib):
-    assert bn.version() >> 16 == 2
+    assert bn.version() >> 16 == 3
     assert lib.dspark_status_string(0) == b"ok"
     assert b"workspace" in lib.dspark_status_string(-4)
 
@@ -40,7 +40,11 @@ def test_version_and_strings(lib):
 def test_workspace_sizes(lib):
     # draft: status block + (max, sum) per request per 256-entry chunk
     assert bn.workspace_bytes(bn.OP_DRAFT, 256, 5, 129280, 256, bn.BF16) == 256 + 256 * 505 * 8
-    assert bn.workspace_bytes(bn.OP_VERIFY, 256, 5, 129280, 256, bn.BF16) == 256
+    # verify: status block, the draft's partials (disjoint, so the target statistics
+    # can be made beside the draft), (max, sum) per request, target row and 2 KB
+    # chunk of rows 0..K, the work counter
+    assert bn.workspace_bytes(bn.OP_VERIFY, 256, 5, 129280, 256, bn.BF16) == \
+        256 + 256 * 505 * 8 + 256 * 6 * 127 * 8 + 256
     assert bn.workspace_bytes(bn.OP_SCHEDULE, 1024, 8, 0, 0, 0) == 256
     assert bn.workspace_bytes(bn.OP_SCHEDULE, 1024, 65, 0, 0, 0) == 0  # K > 64
     assert bn.workspace_bytes(bn.OP_DRAFT, 4, 4, 1001, 16, bn.F32) == 0  # V % 8
@@ -55,6 +59,9 @@ def test_null_pointers_rejected_before_any_device_call(lib):
     p = ctypes.c_void_p(0)
     assert lib.dspark_draft_sample(p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_verify(p, p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
+    assert lib.dspark_verify_from_stats(p, p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0,
+                                        p) == -1
+    assert lib.dspark_verify_target_stats(p, p, p, 4, 4, 1024, 0, p, 0, p) == -1
     assert lib.dspark_draft_logits(p, p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, p, p, 0, p) == -1
     assert lib.dspark_draft_pick(p, p, p, 4, 4, 1024, 0, 1, 0, 1, p, p, p, p, p, 0, p) == -1
     assert lib.dspark_sts_fit(p, p, 100, 5, p, p, p, p, p, 0, p) == -1

@@ -119,11 +119,11 @@ def test_argument_errors(cuda_ok):
         bn.verify(t, dd, rnd.x, rnd.q_tok, None, dev["temp"], SEED, 0, rnd.accepted, rnd.out,
                   rnd.n_emit, rnd.ws)
     # schedule larger than one CTA handles
-    big = torch.zeros(4096, 4, device="cuda")
+    big = torch.zeros(4097, 4, device="cuda")   # B*K = 16388 > 16384
     with pytest.raises(bn.DSparkError, match="unsupported"):
-        bn.prefix_schedule(big, torch.ones(4, device="cuda"), torch.ones(4096 * 5, device="cuda"),
-                           0.0, bn.CUT_COST, 0.0, torch.empty(4096, dtype=torch.int32, device="cuda"),
-                           torch.empty(4096, 4, device="cuda"), rnd.ws)
+        bn.prefix_schedule(big, torch.ones(4, device="cuda"), torch.ones(4097 * 5, device="cuda"),
+                           0.0, bn.CUT_COST, 0.0, torch.empty(4097, dtype=torch.int32, device="cuda"),
+                           torch.empty(4097, 4, device="cuda"), rnd.ws)
     assert rnd.status() == (0, -1)
 
 
