@@ -398,11 +398,21 @@ def main():
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
             round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream, q_norm=rnd.q_norm),
             stream, 20)
+        ms_stats = time_region(lambda: bn.verify_target_stats(
+            dev["target"], rnd.cut, dev["temp"], rnd.ws, stream), stream, 20)
+        ms_final = time_region(lambda: bn.verify_from_stats(
+            dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
+            round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream, q_norm=rnd.q_norm),
+            stream, 20)
 
-    # verify's algorithmic bytes: target rows 0..a_b of every request, plus the
-    # draft row a_b of every request rejected before its cut
+    # verification's algorithmic bytes (the survey's count): target rows 0..cut[b]
+    # of every request, plus draft row a_b of every request rejected before its
+    # cut. The statistics pass reads the former, the final kernel the draft rows
+    # and (again) the target row of the residual.
     rej = int((acc_np < cut).sum())
-    verify_bytes = (int((acc_np + 1).sum()) + rej) * w.V * s_bytes
+    stats_bytes = int((cut + 1).sum()) * w.V * s_bytes
+    final_bytes = 2 * rej * w.V * s_bytes
+    verify_bytes = stats_bytes + rej * w.V * s_bytes
     verify_gbs = verify_bytes / (ms_verify * 1e-3) / 1e9
     # the draft kernel (one cooperative launch per round): per position the
     # base block in, d out, W once, the chunk partials out and back in, the
@@ -457,15 +467,24 @@ def main():
         "emitted_tok_per_s": emit_all * 1000.0 / ms,
         "accepted_per_round": accepted, "emitted_per_round": emitted,
         "mean_cut": float(cut.mean()), "mean_accepted": float(acc_np.mean()),
-        "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify},
+        "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify,
+                      "verify_target_stats": ms_stats, "verify_from_stats": ms_final,
+                      "round_minus_draft": ms - ms_draft},
         "verify": {"gbs": verify_gbs, "frac_of_hbm_peak": verify_gbs / hbm,
-                   "bytes_per_launch": verify_bytes, "launch_ms": ms_verify},
+                   "bytes_per_call": verify_bytes, "call_ms": ms_verify,
+                   "target_stats": {"bytes": stats_bytes, "ms": ms_stats,
+                                    "gbs": stats_bytes / (ms_stats * 1e-3) / 1e9,
+                                    "frac_of_hbm_peak": stats_bytes / (ms_stats * 1e-3) / 1e9 / hbm},
+                   "from_stats": {"bytes": final_bytes, "ms": ms_final,
+                                  "gbs": final_bytes / (ms_final * 1e-3) / 1e9,
+                                  "frac_of_hbm_peak": final_bytes / (ms_final * 1e-3) / 1e9 / hbm},
+                   "bytes_rule": "target rows 0..cut[b] + draft row a_b of each rejected request"},
         "draft_stage": {"gbs": draft_gbs, "bias_gemm_tflops": gemm_tflops,
                         "bias_gemm_frac_of_bf16_peak": gemm_tflops / tflops},
         "roofline": roof,
         "e2e": {"value": world * 1000.0 / ms_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clk,
     }
     if (rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name

@@ -27,6 +27,7 @@ enum WaitSite : unsigned int {
   kWhereTcAccFull = 14,
   kWhereTcAccEmpty = 15,
   kWhereTcGrid = 16,
+  kWhereTcDStore = 17,
   kWhereStatsEmpty = 20,
   kWhereStatsFull = 21,
 };
@@ -162,6 +163,35 @@ struct Elem<DSPARK_BF16> {
     return __bfloat16_as_ushort(__float2bfloat16_rn(v));
   }
   __device__ __forceinline__ static float to_float(T v) { return bf16_bits_to_float(v); }
+};
+
+// 16 bytes of logits (8 bf16 or 4 fp32) as floats in index order, from shared
+// or global memory.
+template <int DT>
+struct Vec16;
+template <>
+struct Vec16<DSPARK_BF16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const void* p, float* v) {
+    const uint4 q = *reinterpret_cast<const uint4*>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  }
+};
+template <>
+struct Vec16<DSPARK_F32> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const void* p, float* v) {
+    const float4 q = *reinterpret_cast<const float4*>(p);
+    v[0] = q.x;
+    v[1] = q.y;
+    v[2] = q.z;
+    v[3] = q.w;
+  }
 };
 
 // 2^x on the special-function unit (ex2.approx; subnormal results flush to

@@ -15,19 +15,22 @@
 // memory (two 256-column buffers).
 //
 // Persistent CTAs, one per SM, warp-specialised:
-//   warp 0     TMA producer of W tiles (ring of four 16 KB stages of 64 ranks x
-//              128 vocabulary entries: one vocabulary half of a tile per four stages)
+//   warp 0     TMA producer of W tiles (ring of six 16 KB stages of 64 ranks x
+//              128 vocabulary entries: a vocabulary half of a tile per four stages)
 //   warp 1     TMEM allocator and the single-thread tcgen05.mma issuer (it
 //              waits at a named barrier for A, which the epilogue warps gather
 //              while the producers already stream W and base)
-//   warp 2     TMA producer of base tiles (ring of six 16 KB [128 x 64] blocks,
-//              so the next tile's blocks load while this one is processed)
+//   warp 2     TMA producer of base tiles (ring of four 16 KB [128 x 64] blocks)
+//              and the TMA store of d from the same slots: a slot is refilled
+//              once its store has read it, so the epilogue never waits on a
+//              store
 //   warps 4-11 epilogue, two halves of four warps (one per TMEM lane
 //              quadrant): half h takes column blocks h and h+2 of every tile.
 //              tcgen05.ld of the accumulator (lane = request row), + base,
-//              round to bf16 (packed), write d back into the staged block, TMA
-//              store of d, running (max, sum exp2) per row; the halves merge
-//              their row statistics through shared memory at the end of a tile.
+//              round to bf16 (packed), write d back into the staged block and
+//              hand it to the producer's store, running (max, sum exp2) per
+//              row; the halves merge their row statistics through shared
+//              memory at the end of a tile.
 // Every wait on an mbarrier is bounded; a CTA that gives up reports
 // DSPARK_STATUS_TIMEOUT and winds down instead of hanging.
 #include <cuda.h>
@@ -46,10 +49,10 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 256;
 constexpr int kWRows = 64;          // Markov ranks per W stage
 constexpr int kWCols = 128;         // vocabulary columns per W stage (one MMA half)
-constexpr int kWStages = 4;         // W ring depth (stages of 64 ranks x 128 vocab)
+constexpr int kWStages = 6;         // W ring depth (stages of 64 ranks x 128 vocab)
 constexpr int kWStageBytes = kWRows * kWCols * 2;
 constexpr int kWBoxBytes = kWRows * 64 * 2;  // one [64 ranks x 64 vocab] TMA box
-constexpr int kBaseSlots = 6;       // base/d ring of [128 x 64] blocks: 1.5 tiles
+constexpr int kBaseSlots = 4;       // base/d ring of [128 x 64] blocks: one tile
 constexpr int kBlockBytes = 128 * 64 * 2;
 constexpr int kABytes = 128 * 256 * 2;  // gathered U rows, 4 k-blocks of [128 x 64]
 
@@ -58,7 +61,7 @@ constexpr int kOffA = 0;
 constexpr int kOffW = kOffA + kABytes;
 constexpr int kOffBase = kOffW + kWStages * kWStageBytes;
 constexpr int kOffBar = kOffBase + kBaseSlots * kBlockBytes;
-constexpr int kNumBars = 2 * kWStages + 2 * kBaseSlots + 6;
+constexpr int kNumBars = 2 * kWStages + 2 * kBaseSlots + 7;
 constexpr int kOffX = kOffBar + kNumBars * 8 + 16;              // [2][128] float2 row stats
 constexpr int kSmemBytes = kOffX + 2 * 128 * 8;
 static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory per block");
@@ -96,6 +99,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* b) {
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t par) {
   return mbar_wait_bounded(su32(b), par);
+}
+// True once the phase of parity `par` has completed (no waiting).
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t par) {
+  uint32_t ok;
+  asm volatile("{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+               : "=r"(ok)
+               : "r"(su32(b)), "r"(par)
+               : "memory");
+  return ok != 0;
 }
 
 // L2 eviction policies: W is re-read by every draft position (keep it), base
@@ -234,9 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* w_full = bars;
   uint64_t* w_empty = bars + kWStages;
   uint64_t* b_full = bars + 2 * kWStages;
-  uint64_t* b_empty = b_full + kBaseSlots;
-  uint64_t* t_full = b_empty + kBaseSlots;   // [2 buffers][2 halves]
+  uint64_t* t_full = b_full + kBaseSlots;    // [2 buffers][2 halves]
   uint64_t* t_empty = t_full + 4;            // [2]
+  uint64_t* d_full = t_empty + 2;            // [kBaseSlots] the block's d is written
+  uint64_t* d_done = d_full + kBaseSlots;    // the position's d stores are complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kNumBars);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
   float2* xstat = reinterpret_cast<float2*>(smem + kOffX);
@@ -260,10 +273,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kBaseSlots; ++i) {
       mbar_init(&b_full[i], 1);
-      mbar_init(&b_empty[i], 1);
+      mbar_init(&d_full[i], 1);
     }
+    mbar_init(d_done, 1);
     for (int i = 0; i < 4; ++i) mbar_init(&t_full[i], 1);
     for (int i = 0; i < 2; ++i) mbar_init(&t_empty[i], 256);
+    // w_full, w_empty, b_full, t_full (4), t_empty (2), d_full, d_done
+    static_assert(2 * kWStages + 2 * kBaseSlots + 7 == kNumBars, "barrier count");
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -324,18 +340,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < kWStages; ++q)
         if (last[q] >= 0) mbar_wait(&w_full[q], (last[q] / kWStages) & 1);
   } else if (warp == 2 && lane == 0) {
-    // ---------------- base producer ----------------
+    // ---------------- base producer and d stores ----------------
     // block j of tile t (counted over all positions) is block g = 4t + j of
-    // the ring (slot g % kBaseSlots)
+    // the ring (slot g % kBaseSlots). The epilogue writes a block's d back
+    // into its slot and arrives on d_full; this thread stores it (in block
+    // order) and refills the slot once the store has read it.
     const uint64_t pol_base = policy_evict_first();
+    // d keeps the normal L2 priority: the sampler re-reads a chunk of every row
+    const uint64_t pol_d = policy_evict_normal();
+    const int total = 4 * n_my * npos;
     int last[kBaseSlots];
     for (int q = 0; q < kBaseSlots; ++q) last[q] = -1;
-    for (int g = 0; g < 4 * n_my * npos; ++g) {
+    int next_store = 0;
+    // 1: block gsb's store issued; 0: its d is not written yet (no wait); -1: gave up
+    auto store_block = [&](int gsb, bool wait) -> int {
+      const int s2 = gsb % kBaseSlots;
+      const uint32_t par = (gsb / kBaseSlots) & 1;
+      if (wait) {
+        if (!mbar_wait(&d_full[s2], par)) return -1;
+      } else if (!mbar_test(&d_full[s2], par)) {
+        return 0;
+      }
+      const int t = gsb >> 2;
+      const int n0 = (nt0 + (t % n_my) * nstride) * kTileN;
+      const int kpos = p.k + t / n_my;
+      tma_store_3d(&map_d, sBase + s2 * kBlockBytes, n0 + (gsb & 3) * 64, kpos - 1, m0, pol_d);
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      if (p.fused && (gsb + 1) % (4 * n_my) == 0) {
+        // the position's last block: its d must be in global memory before
+        // the grid barrier, where the sampler starts reading it
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        mbar_arrive(d_done);
+      }
+      return 1;
+    };
+    bool gave_up = false;
+    for (int g = 0; g < total && !gave_up; ++g) {
       const int s = g % kBaseSlots;
-      if (*(volatile int*)abort_flag || !mbar_wait(&b_empty[s], ((g / kBaseSlots) & 1) ^ 1)) {
-        if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcBaseEmpty, m0);
-        *(volatile int*)abort_flag = 1;
-        break;
+      if (*(volatile int*)abort_flag) break;
+      if (g >= kBaseSlots) {
+        // the slot's previous block (g - kBaseSlots) must be stored and read
+        while (next_store <= g - kBaseSlots) {
+          if (store_block(next_store, true) < 0) {
+            gave_up = true;
+            break;
+          }
+          ++next_store;
+        }
+        if (gave_up) break;
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
       }
       const int t = g >> 2;
       const int n0 = (nt0 + (t % n_my) * nstride) * kTileN;
@@ -343,8 +397,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_expect_tx(&b_full[s], kBlockBytes);
       tma_load_3d(sBase + s * kBlockBytes, &map_base, n0 + (g & 3) * 64, kpos - 1, m0, &b_full[s], pol_base);
       last[s] = g;
+      // blocks whose d is already written go out now
+      while (next_store < g && store_block(next_store, false) == 1) ++next_store;
     }
-    if (*(volatile int*)abort_flag)
+    while (!gave_up && next_store < total && !*(volatile int*)abort_flag) {
+      if (store_block(next_store, true) < 0) gave_up = true;
+      else ++next_store;
+    }
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (gave_up) {
+      if (!*(volatile int*)abort_flag) report_wait(p.status, kWhereTcDStore, m0);
+      *(volatile int*)abort_flag = 1;
+    }
+    if (*(volatile int*)abort_flag)  // let issued loads land before the CTA winds down
       for (int q = 0; q < kBaseSlots; ++q)
         if (last[q] >= 0) mbar_wait(&b_full[q], (last[q] / kBaseSlots) & 1);
   } else if (warp == 1) {
@@ -465,9 +530,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sc = (valid && p.bias_scale) ? p.bias_scale[b] : 1.f;
     const uint32_t lane_base = (uint32_t)(q * 32) << 16;
     const bool elected = (warp == 4 + 4 * h) && lane == 0;
-    // d keeps the normal L2 priority: the sampler re-reads one 256-entry
-    // chunk of every row right after the position ends
-    const uint64_t pol_d = policy_evict_normal();
     bool miss = false;
     bool aborted = false;
     const bool leader = warp == 4 && lane == 0;
@@ -580,24 +642,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_async_smem();
         __syncwarp();
-        half_bar(h);
-        if (elected) {
-          tma_store_3d(&map_d, sBase + slot * kBlockBytes, n0 + j * 64, kpos - 1, m0, pol_d);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          if (jj == 1) {
-            // the first block's store has read its slot: hand it back; the
-            // second block's slot is handed back at the end of the tile
-            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-            mbar_arrive(&b_empty[(4 * ti + h) % kBaseSlots]);
-          }
-        }
-        __syncwarp();  // lane 0 may still be in the store above
+        half_bar(h);  // the half's four warps have written the block
+        if (elected) mbar_arrive(&d_full[slot]);
+        __syncwarp();
       }
-      if (elected) {
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        mbar_arrive(&b_empty[(4 * ti + h + 2) % kBaseSlots]);
-      }
-      __syncwarp();
       // this thread is done reading accumulator buffer `buf`
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       mbar_arrive(&t_empty[buf]);
@@ -637,16 +685,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (!aborted && p.fused) {
       // this position's d is complete in global memory (the sampler reads it)
-      if (elected) {
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
+      // (d_done completes once per position, so this wait is never two phases
+      // behind; a CTA without tiles stores nothing and skips it)
+      bool fail = leader && n_my > 0 && !mbar_wait(d_done, kp & 1);
+      if (fail) report_wait(p.status, kWhereTcDStore, m0);
       __syncwarp();
-      // every CTA's partials and d of this position -> sample -> every token
-      epi_bar_any(false);
-      bool fail = leader && !grid_arrive_wait(p.gbar, (++nbar) * gridDim.x);
-      if (fail) report_wait(p.status, kWhereTcGrid, m0);
       aborted = epi_bar_any(fail);
+      // every CTA's partials and d of this position -> sample -> every token
+      if (!aborted) {
+        fail = leader && !grid_arrive_wait(p.gbar, (++nbar) * gridDim.x);
+        if (fail) report_wait(p.status, kWhereTcGrid, m0);
+        aborted = epi_bar_any(fail);
+      }
       if (!aborted) {
         for (int rr = blockIdx.x + (warp - 4) * gridDim.x; rr < p.B; rr += 8 * gridDim.x)
           sample_row_warp<DSPARK_BF16>(p.da, rr, kpos);
@@ -666,7 +716,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       a_ready_arrive();
     }
     }
-    if (elected) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
   }
 
   __syncwarp();  // role lanes rejoin their warps before the block barrier

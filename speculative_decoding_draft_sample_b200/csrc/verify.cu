@@ -79,34 +79,6 @@ __device__ __forceinline__ uint4 dsmem_load16(const void* local, int rank) {
   return v;
 }
 
-// 16 bytes of shared memory as floats (8 bf16 or 4 fp32), in index order.
-template <int DT>
-struct Vec16;
-template <>
-struct Vec16<DSPARK_BF16> {
-  static constexpr int N = 8;
-  __device__ __forceinline__ static void load(const void* p, float* v) {
-    const uint4 q = *reinterpret_cast<const uint4*>(p);
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[2 * j] = __uint_as_float(w[j] << 16);
-      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
-    }
-  }
-};
-template <>
-struct Vec16<DSPARK_F32> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void load(const void* p, float* v) {
-    const float4 q = *reinterpret_cast<const float4*>(p);
-    v[0] = q.x;
-    v[1] = q.y;
-    v[2] = q.z;
-    v[3] = q.w;
-  }
-};
-
 // Combines the online pair (m2, s2) into (m, s); NaN propagates.
 __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
   const float mm = fmaxf(m, m2);

@@ -43,9 +43,9 @@ def test_zero_recurrence_is_the_markov_head_bit_for_bit():
     rng = np.random.default_rng(1)
     for dtype in ("bf16", "f32", "f64"):
         inp = _inp(6, 4, 64, 8, rng, dtype)
-        if dtype == "bf16":  # factors stored in bf16, as the device reads them
-            inp["U"] = o.round_to_bf16(inp["U"])[0]
-            inp["W"] = o.round_to_bf16(inp["W"])[0]
+        # factors stored in the logits' dtype, as the device reads them
+        inp["U"] = o.round_to_storage(inp["U"], dtype)[0]
+        inp["W"] = o.round_to_storage(inp["W"], dtype)[0]
         mk = o.draft_round(inp, SEED, 3)
         rc = o.draft_round(dict(inp, R=np.zeros((8, 8))), SEED, 3)
         for key in ("d", "x", "q_tok", "q_lse"):
