@@ -307,6 +307,8 @@ def main():
                          "threshold, or none (every request verifies all K drafts)")
     ap.add_argument("--threshold", type=float, default=0.5,
                     help="survival threshold of --cut threshold")
+    ap.add_argument("--head", default="markov", choices=["markov", "recurrent"],
+                    help="sequential draft head: the Markov head (default) or the recurrent one")
     args = ap.parse_args()
     if args.load_sweep:
         load_sweep()
@@ -324,6 +326,8 @@ def main():
 
     # each rank: its own batch (weak scaling), no collective on the data path
     inp = wl.generate(replicas.rank_workload(w, rank))
+    if args.head == "recurrent":
+        inp["R"] = wl.recurrent_factor(w)
     dev = to_device(inp)
     tdt = torch.float32 if w.dtype == wl.F32 else torch.bfloat16
     rnd = SpecRound(w.B, w.K, w.V, w.r, tdt)
@@ -387,10 +391,16 @@ def main():
     # per-stage times (same stream, CUDA events), each stage alone
     s_bytes = w.nbytes_per_logit
     with torch.cuda.stream(stream):
-        ms_draft = time_region(lambda: bn.draft_sample(
-            dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], dev["temp"],
-            wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream,
-            q_norm=rnd.q_norm), stream, 10)
+        if args.head == "recurrent":
+            ms_draft = time_region(lambda: bn.draft_sample_recurrent(
+                dev["base"], dev["U"], dev["W"], dev["R"], dev["bias_scale"], dev["last_tok"],
+                dev["temp"], wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.h,
+                rnd.ws, stream, q_norm=rnd.q_norm), stream, 10)
+        else:
+            ms_draft = time_region(lambda: bn.draft_sample(
+                dev["base"], dev["U"], dev["W"], dev["bias_scale"], dev["last_tok"], dev["temp"],
+                wl.PHILOX_SEED, round_id, rnd.x, rnd.d, rnd.q_lse, rnd.q_tok, rnd.ws, stream,
+                q_norm=rnd.q_norm), stream, 10)
         ms_sched = time_region(lambda: bn.prefix_schedule(
             dev["conf_logit"], dev["pos_temp"], dev["step_cost"], dev["fixed_cost"], mode,
             threshold, rnd.cut, rnd.survival, rnd.ws, stream), stream, 20)
@@ -442,8 +452,8 @@ def main():
 
     in_bytes = (w.B * (w.K + 1) * w.V + w.B * w.K * w.V + 2 * w.V * w.r) * s_bytes
     traffic, traffic_src = profiled_traffic(DRAFT_KERNEL_SOURCES, "draft_logits_tc_dspark5.txt")
-    if w.name != wl.DSPARK5.name or mode != bn.CUT_COST:
-        traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload (cost cut) only"
+    if w.name != wl.DSPARK5.name or mode != bn.CUT_COST or args.head != "markov":
+        traffic, traffic_src = None, "ncu summary covers the DSpark-5 workload (cost cut, Markov head) only"
     roof = {"kernel": "draft_logits_tc (dspark_draft_sample: all K positions in one launch)",
             "bound": "hbm", "achieved": draft_gbs, "peak": hbm, "unit": "GB/s",
             "frac": draft_gbs / hbm, "traffic": traffic, "traffic_source": traffic_src,
@@ -459,6 +469,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
                    "global_batch": w.B * world, "parallelism": f"replicas{world}",
                    "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else ""),
+                   "head": args.head,
                    "l2": (f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2 (126 MB); not flushed"
                           if in_bytes > L2_BYTES else
                           f"inputs ({in_bytes / 1e6:.0f} MB) fit in L2 (126 MB); not flushed"),
@@ -488,7 +499,7 @@ def main():
         "clocks": clk,
     }
     if (rank == 0 and world == 1 and not args.no_cpu_baseline and w.name == wl.DSPARK5.name
-            and mode == bn.CUT_COST):
+            and mode == bn.CUT_COST and args.head == "markov"):
         line["cpu_baseline"] = {k: v for k, v in cpu_baseline(w, wl.small_inputs(w), ORACLE_SAMPLE,
                                                               0).items()
                                 if k in ("value", "unit", "cores", "blas_threads", "kind", "sample")}

@@ -5,7 +5,8 @@
  *   dspark_draft_sample    semi-autoregressive draft: parallel base logits plus
  *                          a low-rank Markov-head bias, sampled position by position
  *                          (dspark_draft_logits / dspark_draft_pick: one position's
- *                          two halves)
+ *                          two halves; dspark_draft_sample_recurrent: the recurrent
+ *                          head in place of the Markov head)
  *   dspark_prefix_schedule calibrated confidence, survival products and the
  *                          early-stopping prefix cut against a cost-per-token table
  *   dspark_sts_fit         Sequential Temperature Scaling of the confidences, ECE
@@ -130,6 +131,33 @@ int dspark_draft_sample(const void* base, const void* U, const void* W,
                         uint64_t seed, uint64_t round_id, int32_t* x, void* d,
                         float* q_lse, float* q_tok, float* q_norm, void* ws,
                         size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * dspark_draft_sample with the recurrent sequential head in place of the
+ * Markov head. [P1] "DSpark's semi-autoregressive compromise" (recurrent head
+ * machinery beside the Markov head); [P3] "The Semi-Autoregressive Trick" (an
+ * optional head that tracks the full block prefix, with marginal gains). The
+ * pages give no equations; this library's reading is a state h_k in R^r with
+ *   h_1 = U[x_0],  h_k = round_dtype(U[x_{k-1}] + tanh(h_{k-1} @ R))  (k >= 2)
+ *   bias_k = bias_scale[b] * h_k @ W
+ * (fp32 accumulation in ascending order of the rank index, tanh in fp32), so
+ * that R = 0 gives dspark_draft_sample's results bit for bit, while a non-zero
+ * R lets position k depend on every earlier token of the block.
+ *
+ *   R   [r, r] dtype   the state matrix (row j multiplies h_j)
+ *   h   [B, K, r] dtype out   the states h_1..h_K of every request
+ * Every other argument, output and limit as for dspark_draft_sample; r must
+ * also be a multiple of 8, and R and h 16-byte aligned. The draw of position k
+ * forms h_{k+1} in the same launch (one warp per request: about r^2 multiply-
+ * adds and r tanh evaluations).
+ */
+int dspark_draft_sample_recurrent(const void* base, const void* U, const void* W,
+                                  const void* R, const float* bias_scale,
+                                  const int32_t* last_tok, const float* temp, int B,
+                                  int K, int V, int r, int dtype, uint64_t seed,
+                                  uint64_t round_id, int32_t* x, void* d, float* q_lse,
+                                  float* q_tok, float* q_norm, void* h, void* ws,
+                                  size_t ws_bytes, dspark_stream_t stream);
 
 /*
  * The two halves of one draft position of dspark_draft_sample, for callers
@@ -318,7 +346,9 @@ int dspark_sts_fit(const float* conf_logit, const uint8_t* survived, int N, int 
  * image, held on every GPU that loads the library until the process exits; the
  * call allocates and frees nothing. Its device address is looked up once per
  * device, by the first call made while that device is current, so that first
- * call should come before any stream capture. Every call uses the same array
+ * call should come before any stream capture. The address is kept for the
+ * life of the process: calls after a cudaDeviceReset (or from another CUDA
+ * context on the same device) are not supported. Every call uses the same array
  * and clears its status part first: calls that overlap on the GPU (other
  * streams, other threads) race and must not be issued. A call needs
  * 256 + 8 * B * ceil(V / 256) bytes of the 8 MiB (B = 1024 at V = 151936 takes

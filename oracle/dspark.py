@@ -155,26 +155,41 @@ def recurrent_state(U: np.ndarray, R: np.ndarray, prev: np.ndarray, h_prev: np.n
 
     Returns (h [B, r], flag [B, r]). For bf16 storage an element is flagged
     when its fp64 value lies within the error of a device computing it in fp32
-    of a rounding midpoint: the fp32 accumulation of r products (r 2^-23
-    sum_j |h_j R_ji|), tanh to 2^-22 relative, and the final fp32 add
-    (2^-22 |v|).
+    of a rounding midpoint. The device sums h_j R_ji with fused multiply-adds
+    in ascending j, each rounding its partial sum once, so its error in a is
+    at most 2^-24 sum_j |S_j| to first order (S_j the exact partial sums in
+    that order); tanh adds 2^-22 |tanh a| (two units in the last place; its
+    slope is at most 1, so the error in a passes through unamplified) and the
+    final add 2^-23 |v|.
     """
     U = np.asarray(U, np.float64)
     R = np.asarray(R, np.float64)
     h_prev = np.asarray(h_prev, np.float64)
+    h, flag, _ = recurrent_state_window(U, R, prev, h_prev, dtype)
+    return h, flag
+
+
+def recurrent_state_window(U: np.ndarray, R: np.ndarray, prev: np.ndarray, h_prev: np.ndarray,
+                           dtype: str):
+    """``recurrent_state`` plus the error window of every element (the bound
+    above, in absolute terms). For fp32 storage there is no rounding point to
+    flag: every element is returned flagged, and a check compares a device's
+    state with this one within the window instead."""
     a = h_prev @ R
     th = np.tanh(a)
     v = U[np.asarray(prev, np.int64)] + th
+    partial = np.cumsum(h_prev[:, :, None] * R[None, :, :], axis=1)   # [B, j, i]
+    acc_err = 2.0 ** -24 * np.abs(partial).sum(axis=1)
+    win = acc_err + 2.0 ** -22 * np.abs(th) + 2.0 ** -23 * np.abs(v)
     if dtype != "bf16":
-        return round_to_storage(v, dtype)
-    r = R.shape[0]
+        out, _ = round_to_storage(v, dtype)
+        return out, np.ones(np.shape(v), bool), win + 2.0 ** -24 * np.abs(v)
     m, e = np.frexp(v)
     sc = m * 256.0
     out = np.ldexp(np.rint(sc), e - 8)
     mid = np.ldexp(np.trunc(sc) + np.sign(sc) * 0.5, e - 8)
-    win = 2.0 ** -22 * (np.abs(v) + np.abs(th)) + r * 2.0 ** -23 * (np.abs(h_prev) @ np.abs(R))
     flag = np.isfinite(v) & (np.abs(v - mid) <= win)
-    return out, flag
+    return out, flag, win
 
 
 def inverse_cdf(w: np.ndarray, u: np.ndarray, window: float = U_WINDOW, normalized: bool = True):
@@ -274,7 +289,8 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
     Teacher forcing: with ``teacher`` (the GPU's "d" [B,K,V] and "x" [B,K],
     and "h" [B,K,r] for the recurrent head), a flagged d or h element takes
     the teacher's value and a flagged draw takes the teacher's token;
-    ``forced`` counts how often that changed anything.
+    ``forced`` counts how often that changed a logit or a token, ``h_forced``
+    how many state elements were adopted.
     """
     base = inp["base"]
     B, K, V = base.shape
@@ -292,18 +308,21 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
     r = np.shape(inp["U"])[1]
     hs = np.zeros((B, K, r)) if Rm is not None else None
     h_flag = np.zeros((B, K), bool)
+    h_forced = 0
+    h_excess = 0.0  # fp32 states: the largest amount by which a device state leaves its window
     h = np.zeros((B, r))
     for k in range(1, K + 1):
         u = uniform(seed, req, k, PURPOSE_DRAFT, round_id)
         if Rm is not None:
-            h, hf = recurrent_state(inp["U"], Rm, prev, h, inp["dtype"])
+            h, hf, hwin = recurrent_state_window(inp["U"], Rm, prev, h, inp["dtype"])
             if teacher is not None and hf.any():
                 th = np.asarray(teacher["h"][:, k - 1], np.float64)
-                diff = hf & (th != h)
-                forced += int(diff.sum())
+                if inp["dtype"] != "bf16":  # no rounding point: the device's state within the window
+                    h_excess = max(h_excess, float((np.abs(th - h) - hwin).max()))
+                h_forced += int((hf & (th != h)).sum())
                 h = np.where(hf, th, h)
             hs[:, k - 1] = h
-            h_flag[:, k - 1] = hf.any(axis=1)
+            h_flag[:, k - 1] = hf.any(axis=1) if inp["dtype"] == "bf16" else False
         st = draft_position(base[:, k - 1], inp["U"], inp["W"], prev, inp["bias_scale"],
                             tau, u, inp["dtype"], h if Rm is not None else None)
         if teacher is not None and st["d_flag"].any():
@@ -332,7 +351,7 @@ def draft_round(inp: Dict[str, np.ndarray], seed: int, round_id: int,
         x_flag[:, k - 1] = st["x_flag"]
         prev = st["x"]
     return dict(d=d, d_flag=d_flag, x=x, q_lse=q_lse, q_tok=q_tok, x_flag=x_flag,
-                h=hs, h_flag=h_flag, forced=forced)
+                h=hs, h_flag=h_flag, h_forced=h_forced, h_excess=h_excess, forced=forced)
 
 
 # --------------------------------------------------------------------------

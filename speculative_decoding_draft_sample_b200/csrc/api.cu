@@ -167,6 +167,8 @@ int draft_prepare(DraftArgs& a, int* sms, bool logits, bool pick, const void* ba
   a.status = static_cast<Status*>(ws);
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(ws) + kStatusBytes);
   a.nchunk = nchunks(V);
+  a.R = nullptr;  // the Markov head unless the caller adds the recurrent one
+  a.H = nullptr;
   return DSPARK_OK;
 }
 
@@ -192,6 +194,33 @@ int dspark_draft_sample(const void* base, const void* U, const void* W, const fl
   // one cooperative launch for the whole block when the tensor-core path
   // applies and every M-tile gets its own CTAs; otherwise two launches per
   // position (the same kernels, so the results are identical)
+  if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, s));
+  for (int k = 1; k <= K; ++k) {
+    cudaError_t e = launch_logits(a, k, sms, s);
+    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  return DSPARK_OK;
+}
+
+int dspark_draft_sample_recurrent(const void* base, const void* U, const void* W, const void* R,
+                                  const float* bias_scale, const int32_t* last_tok,
+                                  const float* temp, int B, int K, int V, int r, int dtype,
+                                  uint64_t seed, uint64_t round_id, int32_t* x, void* d,
+                                  float* q_lse, float* q_tok, float* q_norm, void* h, void* ws,
+                                  size_t ws_bytes, dspark_stream_t stream) {
+  if (!R || !h) return DSPARK_ERR_INVALID_ARG;
+  if (!aligned16(R) || !aligned16(h) || r % 8 != 0) return DSPARK_ERR_INVALID_ARG;
+  DraftArgs a;
+  int sms = 0;
+  if (int e = draft_prepare(a, &sms, true, true, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
+                            dtype, seed, round_id, x, d, q_lse, q_tok, q_norm, ws, ws_bytes))
+    return e;
+  a.R = R;
+  a.H = h;
+  cudaStream_t s = (cudaStream_t)stream;
+  // the same launches as dspark_draft_sample; the draw of every position also
+  // forms the next position's state, and the bias rows come from the states
   if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, s));
   for (int k = 1; k <= K; ++k) {
     cudaError_t e = launch_logits(a, k, sms, s);

@@ -42,10 +42,10 @@ __global__ void __launch_bounds__(256) draft_logits_simt(DraftArgs a, int k) {
   const int b0 = blockIdx.y * BT;
   const int v = chunk * kChunk + tid;
   const bool col_ok = v < a.V;
-  const T* U = static_cast<const T*>(a.U);
   const T* W = static_cast<const T*>(a.W);
 
-  // gather U rows of the previous tokens
+  // gather U rows of the previous tokens (or the recurrent head's states);
+  // the recurrent head's first states h_1 = U[x_0] are written out once
   for (int i = tid; i < BT * a.r; i += 256) {
     const int bb = i / a.r, j = i - bb * a.r;
     const int b = b0 + bb;
@@ -53,7 +53,9 @@ __global__ void __launch_bounds__(256) draft_logits_simt(DraftArgs a, int k) {
     if (b < a.B) {
       int prev = (k == 1) ? a.last_tok[b] : a.x[(long long)b * a.K + (k - 2)];
       if (prev < 0 || prev >= a.V) prev = 0;  // reported by draft_sample / host checks
-      val = E::load(U, (long long)prev * a.r + j);
+      const T* row = a_row<T>(a, b, k, prev);
+      val = E::load(row, j);
+      if (a.R && k == 1 && blockIdx.x == 0) static_cast<T*>(a.H)[(long long)b * a.K * a.r + j] = row[j];
     }
     us[i] = val;
   }
@@ -163,7 +165,10 @@ __global__ void __launch_bounds__(256) draft_logits_simt(DraftArgs a, int k) {
 template <int DT>
 __global__ void __launch_bounds__(256) draft_sample(DraftArgs a, int k) {
   const int b = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (b < a.B) sample_row_warp<DT>(a, b, k);
+  if (b < a.B) {
+    sample_row_warp<DT>(a, b, k);
+    if (a.R && k < a.K) rnn_step<DT>(a, b, k);  // the recurrent head's next state
+  }
 }
 
 // ---------------------------------------------------------------------------

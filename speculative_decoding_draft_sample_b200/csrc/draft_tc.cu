@@ -491,7 +491,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue warp e gathers rows 16e .. 16e + 15: lanes 0-15 read the rows'
     // tokens, then every lane loads one 16-byte chunk of each of the 16 rows
     // (all loads in flight at once; a row is one 512-byte coalesced read).
-    auto gather_a = [&](const int32_t* prev, int prev_stride) {
+    // Position kq's rows come from U by token, or (recurrent head, kq >= 2)
+    // from the states the draw left in H; the first states h_1 = U[x_0] are
+    // written out by the M-tile's first CTA.
+    auto gather_a = [&](const int32_t* prev, int prev_stride, int kq) {
       const int ew = warp - 4;
       int tokv = 0;
       if (lane < 16) {
@@ -499,14 +502,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (b < p.B) tokv = prev[(long long)b * prev_stride];
         if (tokv < 0 || tokv >= p.V) tokv = 0;  // reported by the sampler
       }
-      const uint16_t* U = static_cast<const uint16_t*>(p.U);
       uint4 v[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int tok = __shfl_sync(0xffffffffu, tokv, i);
+        const int bq = m0 + ew * 16 + i;
         v[i] = make_uint4(0, 0, 0, 0);
-        if (m0 + ew * 16 + i < p.B && lane * 8 < p.r)
-          v[i] = *reinterpret_cast<const uint4*>(U + (long long)tok * p.r + lane * 8);
+        if (bq < p.B && lane * 8 < p.r)
+          v[i] = *reinterpret_cast<const uint4*>(a_row<uint16_t>(p.da, bq, kq, tok) + lane * 8);
+      }
+      if (p.da.R && kq == 1 && nt0 == 0) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int bq = m0 + ew * 16 + i;
+          if (bq < p.B && lane * 8 < p.r)
+            *reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.da.H) + (long long)bq * p.da.K * p.r + lane * 8) = v[i];
+        }
       }
       const int kb = lane >> 3, c = lane & 7;
 #pragma unroll
@@ -516,7 +527,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
     };
-    gather_a(p.prev, p.prev_stride);
+    // The recurrent head's next states h_{kq+1} of the rows this CTA drew at
+    // position kq, by its 256 epilogue threads (thread t: output t): R goes
+    // through the A buffer, which holds nothing between the position's last
+    // MMA and the next gather, in halves of 128 rows; up to four drawn rows'
+    // states h_kq at a time sit in the row-statistics buffer. The sums run in
+    // ascending j with one fused multiply-add per term, as in rnn_step, so the
+    // states are those of the per-position path bit for bit.
+    auto rnn_cta = [&](int kq) {
+      const int et = tid - 128;  // epilogue thread 0..255
+      const int r = p.r;
+      const int K = p.da.K;
+      const uint16_t* Rm = static_cast<const uint16_t*>(p.da.R);
+      const uint16_t* Um = static_cast<const uint16_t*>(p.da.U);
+      uint16_t* Hm = static_cast<uint16_t*>(p.da.H);
+      uint16_t* sR = reinterpret_cast<uint16_t*>(sA);      // [128][r]
+      uint16_t* sh = reinterpret_cast<uint16_t*>(xstat);   // [4][256]
+      for (int w0 = 0; w0 < 8; w0 += 4) {
+        int rows[4];
+        int nr = 0;
+        for (int g = 0; g < 4; ++g) {
+          const int rr = blockIdx.x + (w0 + g) * gridDim.x;
+          rows[g] = rr < p.B ? rr : -1;
+          if (rr < p.B) ++nr;
+        }
+        if (nr == 0) break;
+        epi_bar_any(false);  // the statistics buffer and the A buffer are free
+        for (int i = et; i < 4 * r; i += 256) {
+          const int g = i / r, j = i - g * r;
+          sh[g * 256 + j] = rows[g] >= 0 ? Hm[((long long)rows[g] * K + (kq - 1)) * r + j] : (uint16_t)0;
+        }
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int j0 = 0; j0 < r; j0 += 128) {
+          const int jn = min(128, r - j0);
+          epi_bar_any(false);
+          for (int v = et; v < jn * r / 8; v += 256)  // 16-byte pieces of R rows j0 .. j0 + jn - 1
+            reinterpret_cast<uint4*>(sR)[v] = reinterpret_cast<const uint4*>(Rm + (long long)j0 * r)[v];
+          epi_bar_any(false);
+          if (et < r) {
+            for (int j = 0; j < jn; ++j) {
+              const float rv = bf16_bits_to_float(sR[j * r + et]);
+#pragma unroll
+              for (int g = 0; g < 4; ++g) acc[g] = fmaf(bf16_bits_to_float(sh[g * 256 + j0 + j]), rv, acc[g]);
+            }
+          }
+        }
+        if (et < r) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            if (rows[g] < 0) continue;
+            int tok = p.da.x[(long long)rows[g] * K + (kq - 1)];
+            if (tok < 0 || tok >= p.V) tok = 0;  // reported by the draw
+            const float u = bf16_bits_to_float(Um[(long long)tok * r + et]);
+            Hm[((long long)rows[g] * K + kq) * r + et] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(u + tanhf(acc[g])));
+          }
+        }
+      }
+      epi_bar_any(false);  // A is free for the gather
+    };
+    gather_a(p.prev, p.prev_stride, p.k);
     a_ready_arrive();
     // ---------------- epilogue ----------------
     const int q = warp & 3;             // TMEM lane quadrant
@@ -700,6 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!aborted) {
         for (int rr = blockIdx.x + (warp - 4) * gridDim.x; rr < p.B; rr += 8 * gridDim.x)
           sample_row_warp<DSPARK_BF16>(p.da, rr, kpos);
+        if (p.da.R && kpos < p.da.K) rnn_cta(kpos);
         if (kp + 1 < npos) {
           epi_bar_any(false);
           fail = leader && !grid_arrive_wait(p.gbar, (++nbar) * gridDim.x);
@@ -712,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (kp + 1 < npos) {
       // A of the next position from this position's tokens; on a failure the
       // MMA warp still gets its arrival (it then sees the abort flag)
-      if (!aborted) gather_a(p.da.x + kpos - 1, p.da.K);
+      if (!aborted) gather_a(p.da.x + kpos - 1, p.da.K, kpos + 1);
       a_ready_arrive();
     }
     }

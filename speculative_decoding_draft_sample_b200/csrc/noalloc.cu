@@ -117,6 +117,8 @@ extern "C" int dspark_draft_sample_static(const void* base, const void* U, const
   a.q_tok = q_tok;
   a.q_norm = nullptr;
   a.status = static_cast<Status*>(scratch);
+  a.R = nullptr;  // the Markov head
+  a.H = nullptr;
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(scratch) + kStatusBytes);
   a.nchunk = nchunk;
   const bool tc = draft_tc_supported(a);

@@ -227,4 +227,51 @@ __device__ __forceinline__ void sample_row_warp(const DraftArgs& a, int b, int k
   }
 }
 
+// The recurrent head's next state, by the warp that drew x_k of request b
+// ("DSpark turns speculation into a scheduler", "DSpark's semi-autoregressive
+// compromise": recurrent head machinery beside the Markov head; "DSpark LLM
+// inference speedup", "The Semi-Autoregressive Trick": a head that tracks the
+// whole block prefix): h_{k+1} = round(U[x_k] + tanh(h_k @ R)), read from row
+// k-1 and written to row k of H. Lane l computes the eight outputs
+// i0 + 8l .. i0 + 8l + 7 with fp32 fused multiply-adds in ascending j (r % 8 == 0).
+template <int DT>
+__device__ void rnn_step(const DraftArgs& a, int b, int k) {
+  using E = Elem<DT>;
+  using T = typename E::T;
+  const int lane = threadIdx.x & 31;
+  __syncwarp();  // x_k was written by one lane of this warp
+  int tok = a.x[(long long)b * a.K + (k - 1)];
+  if (tok < 0 || tok >= a.V) tok = 0;  // reported by the draw
+  const int r = a.r;
+  const T* hp = static_cast<const T*>(a.H) + ((long long)b * a.K + (k - 1)) * r;
+  const T* Rm = static_cast<const T*>(a.R);
+  const T* u = static_cast<const T*>(a.U) + (long long)tok * r;
+  T* hn = static_cast<T*>(a.H) + ((long long)b * a.K + k) * r;
+  for (int i0 = 0; i0 < r; i0 += 256) {
+    const int i = i0 + 8 * lane;
+    const bool on = i < r;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < r; ++j) {
+      const float hj = E::load(hp, j);  // the same address in every lane
+      if (on) {
+        float rv[8];
+        Vec16<DT>::load(Rm + (long long)j * r + i, rv);
+        if (DT == DSPARK_F32) Vec16<DT>::load(Rm + (long long)j * r + i + 4, rv + 4);
+#pragma unroll
+        for (int m = 0; m < 8; ++m) acc[m] = fmaf(hj, rv[m], acc[m]);
+      }
+    }
+    if (on) {
+      float uv[8];
+      Vec16<DT>::load(u + i, uv);
+      if (DT == DSPARK_F32) Vec16<DT>::load(u + i + 4, uv + 4);
+      T out[8];
+#pragma unroll
+      for (int m = 0; m < 8; ++m) out[m] = E::store_round(uv[m] + tanhf(acc[m]));
+#pragma unroll
+      for (int m = 0; m < 8; ++m) hn[i + m] = out[m];
+    }
+  }
+}
+
 }  // namespace dspark

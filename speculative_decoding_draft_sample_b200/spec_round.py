@@ -28,6 +28,7 @@ class SpecRound:
         self.q_lse = torch.empty((B, K), **f32)
         self.q_tok = torch.empty((B, K), **f32)
         self.q_norm = torch.empty((B, K, 2), **f32)  # the draws' normalisers, for verify
+        self.h = None  # the recurrent head's states [B, K, r], when a round uses it
         self.cut = torch.empty((B,), **i32)
         self.survival = torch.empty((B, K), **f32)
         self.accepted = torch.empty((B,), **i32)
@@ -68,9 +69,17 @@ class SpecRound:
             side_stream.wait_event(fork)
             schedule_and_stats(side_stream)
             join.record(side_stream)
-        bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
-                        inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
-                        self.ws, main, q_norm=self.q_norm)
+        if inp.get("R") is not None:  # the recurrent head; its states land in self.h
+            if self.h is None:
+                self.h = torch.empty((self.B, self.K, self.r), dtype=self.dtype, device=self.x.device)
+            bn.draft_sample_recurrent(inp["base"], inp["U"], inp["W"], inp["R"],
+                                      inp.get("bias_scale"), inp["last_tok"], inp["temp"], seed,
+                                      round_id, self.x, self.d, self.q_lse, self.q_tok, self.h,
+                                      self.ws, main, q_norm=self.q_norm)
+        else:
+            bn.draft_sample(inp["base"], inp["U"], inp["W"], inp.get("bias_scale"), inp["last_tok"],
+                            inp["temp"], seed, round_id, self.x, self.d, self.q_lse, self.q_tok,
+                            self.ws, main, q_norm=self.q_norm)
         if side_stream is None:
             schedule_and_stats(main)
         else:
@@ -85,6 +94,7 @@ class SpecRound:
 
 DEVICE_KEYS = ("base", "target", "U", "W", "bias_scale", "last_tok", "temp", "conf_logit",
                "pos_temp", "step_cost")
+OPTIONAL_KEYS = ("R",)  # the recurrent head's state matrix
 
 
 def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -> Dict[str, object]:
@@ -99,6 +109,11 @@ def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -
             t = t.float()
         t = t.contiguous()
         out[k] = t.pin_memory() if pin else t.to(device, non_blocking=False)
+    for k in OPTIONAL_KEYS:
+        v = inp.get(k)
+        if v is not None:
+            t = v if isinstance(v, torch.Tensor) else torch.from_numpy(v)
+            out[k] = t.contiguous().pin_memory() if pin else t.contiguous().to(device)
     out["fixed_cost"] = float(inp["fixed_cost"])
     return out
 

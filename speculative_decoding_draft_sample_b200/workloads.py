@@ -202,6 +202,15 @@ def small_inputs(w: Workload) -> Dict[str, object]:
                 independent=kinds["independent"])
 
 
+def recurrent_factor(w: Workload, std: float = 1.0) -> torch.Tensor:
+    """A seeded state matrix R [r, r] for the recurrent head, N(0, std^2), in
+    the workload's storage dtype. With U ~ N(0, uw_std^2) the pre-activation
+    h @ R of the first states has std sqrt(r) * uw_std * std (0.8 at r = 256,
+    uw_std = 0.05, std = 1): tanh neither linear nor saturated."""
+    rng = np.random.default_rng([w.seed, 17])
+    return _to_storage(rng.standard_normal((w.r, w.r), dtype=np.float32) * np.float32(std), w.dtype)
+
+
 def generate(w: Workload, requests: Optional[List[int]] = None) -> Dict[str, object]:
     """The full round's inputs (CPU tensors in storage dtype), or only ``requests``' rows.
 

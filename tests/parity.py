@@ -46,8 +46,9 @@ def oracle_inputs(w: wl.Workload, inp: Dict[str, object], requests: List[int]) -
     rows = [pos[b] for b in requests]
     req = np.asarray(requests, np.int64)
     f = lambda t: t.double().numpy()
+    extra = {} if inp.get("R") is None else dict(R=f(inp["R"]))
     return dict(target=f(inp["target"][rows]), base=f(inp["base"][rows]), U=f(inp["U"]),
-                W=f(inp["W"]), last_tok=np.asarray(inp["last_tok"])[req],
+                W=f(inp["W"]), **extra, last_tok=np.asarray(inp["last_tok"])[req],
                 bias_scale=np.asarray(inp["bias_scale"], np.float64)[req],
                 temp=np.asarray(inp["temp"], np.float64)[req],
                 conf_logit=np.asarray(inp["conf_logit"], np.float64),
@@ -60,7 +61,8 @@ def gpu_outputs(rnd: SpecRound, requests: List[int]) -> Dict[str, np.ndarray]:
     idx = torch.as_tensor(requests, device=rnd.x.device, dtype=torch.long)
     a = rnd.accepted[idx].cpu().numpy().astype(np.int64)
     out = rnd.out[idx].cpu().numpy().astype(np.int64)
-    return dict(x=rnd.x[idx].cpu().numpy().astype(np.int64),
+    h = None if rnd.h is None else rnd.h[idx].double().cpu().numpy()
+    return dict(h=h, x=rnd.x[idx].cpu().numpy().astype(np.int64),
                 d=rnd.d[idx].double().cpu().numpy(),
                 q_lse=rnd.q_lse[idx].double().cpu().numpy(),
                 q_tok=rnd.q_tok[idx].double().cpu().numpy(),
@@ -75,10 +77,17 @@ def check_round(w: wl.Workload, inp: Dict[str, object], rnd: SpecRound, requests
     """Teacher-forced parity of every stage on ``requests``; returns counts."""
     g = gpu_outputs(rnd, requests)
     oi = oracle_inputs(w, inp, requests)
-    teacher = dict(d=g["d"], x=g["x"], L=g["L"], a=g["a"], y=g["y"])
+    teacher = dict(d=g["d"], x=g["x"], L=g["L"], a=g["a"], y=g["y"], h=g["h"])
     thr = float(np.float32(threshold))
     r = o.run_round(oi, SEED, round_id, mode, thr, teacher=teacher)
     dr = r["draft"]
+    # the recurrent head's states: exact in bf16 outside flagged elements (the
+    # oracle adopted the GPU's state there), fp32 within rounding of tanh
+    if g["h"] is not None:
+        if w.dtype == wl.BF16:
+            assert np.array_equal(dr["h"], g["h"]), "recurrent states differ outside flagged points"
+        else:  # each fp32 state from the device's previous one, within fp32 error
+            assert dr["h_excess"] <= 0.0, dr["h_excess"]
     # draft: stored logits, tokens, normalisers
     if w.dtype == wl.BF16:
         assert np.array_equal(dr["d"], g["d"]), "stored draft logits differ outside flagged points"
@@ -97,7 +106,9 @@ def check_round(w: wl.Workload, inp: Dict[str, object], rnd: SpecRound, requests
     assert np.array_equal(vr["a"], g["a"]), "accepted lengths differ"
     assert np.array_equal(vr["out"], g["out"]), "emitted tokens differ"
     assert np.array_equal(vr["n_emit"], g["n_emit"])
-    return dict(forced=int(r["forced"]), cut_flag=bool(r["cut_flag"]),
+    return dict(forced=int(r["forced"]), h_flags=int(dr["h_flag"].sum()),
+                h_forced=int(dr["h_forced"]) if w.dtype == wl.BF16 else 0,
+                cut_flag=bool(r["cut_flag"]),
                 cut_forced=int(r["cut_forced"]), d_flags=int(dr["d_flag"].sum()),
                 x_flags=int(dr["x_flag"].sum()), acc_flags=int(vr["acc_flag"].sum()),
                 y_flags=int(vr["y_flag"].sum()), accepted=int(g["a"].sum()))
