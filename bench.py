@@ -481,6 +481,9 @@ def main():
         "stages_ms": {"draft": ms_draft, "schedule": ms_sched, "verify": ms_verify,
                       "verify_target_stats": ms_stats, "verify_from_stats": ms_final,
                       "round_minus_draft": ms - ms_draft},
+        # each stage above alone; in the round the draft leaves this many SMs to
+        # the schedule and the target statistics on the side stream
+        "round_draft_free_sms": rnd.free_sms,
         "verify": {"gbs": verify_gbs, "frac_of_hbm_peak": verify_gbs / hbm,
                    "bytes_per_call": verify_bytes, "call_ms": ms_verify,
                    "target_stats": {"bytes": stats_bytes, "ms": ms_stats,

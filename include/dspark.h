@@ -6,7 +6,8 @@
  *                          a low-rank Markov-head bias, sampled position by position
  *                          (dspark_draft_logits / dspark_draft_pick: one position's
  *                          two halves; dspark_draft_sample_recurrent: the recurrent
- *                          head in place of the Markov head)
+ *                          head in place of the Markov head; dspark_draft_sample_beside:
+ *                          either head, leaving SMs to other streams)
  *   dspark_prefix_schedule calibrated confidence, survival products and the
  *                          early-stopping prefix cut against a cost-per-token table
  *   dspark_sts_fit         Sequential Temperature Scaling of the confidences, ECE
@@ -158,6 +159,40 @@ int dspark_draft_sample_recurrent(const void* base, const void* U, const void* W
                                   uint64_t round_id, int32_t* x, void* d, float* q_lse,
                                   float* q_tok, float* q_norm, void* h, void* ws,
                                   size_t ws_bytes, dspark_stream_t stream);
+
+/*
+ * dspark_draft_sample (R == NULL) or dspark_draft_sample_recurrent (R and h
+ * given) for a caller that runs other work on another stream at the same time.
+ * [P1] "DSpark turns speculation into a scheduler", intro and "Caveats" (the
+ * verifier's pass over the target rows is the other large cost of a round; it
+ * needs only the target logits and the cut, so it can run beside the draft).
+ *
+ * The whole-block launch of dspark_draft_sample (tensor-core path: bf16,
+ * r % 16 == 0, r <= 256, ceil(B / 128) + 2 <= SMs) takes one CTA per SM and
+ * leaves 2 SMs free; this call leaves free_sms SMs free instead (clamped so
+ * that each group of 128 requests keeps at least one SM), for kernels of other
+ * streams such as dspark_verify_target_stats. Fewer CTAs means more vocabulary
+ * tiles per CTA, so the draft itself takes longer; the results are identical
+ * bit for bit to dspark_draft_sample's (or the recurrent call's) for every
+ * free_sms. On the other paths (two launches per position) free_sms has no
+ * effect.
+ *
+ *   R        [r, r] dtype or NULL   the recurrent head's state matrix; NULL
+ *                                   selects the Markov head
+ *   h        [B, K, r] dtype out    the recurrent states (only with R; may be
+ *                                   NULL otherwise)
+ *   free_sms >= 0                   SMs to leave free
+ * Every other argument, output and limit as for dspark_draft_sample; with R
+ * as for dspark_draft_sample_recurrent. DSPARK_ERR_INVALID_ARG for a negative
+ * free_sms.
+ */
+int dspark_draft_sample_beside(const void* base, const void* U, const void* W, const void* R,
+                               const float* bias_scale, const int32_t* last_tok,
+                               const float* temp, int B, int K, int V, int r, int dtype,
+                               uint64_t seed, uint64_t round_id, int32_t* x, void* d,
+                               float* q_lse, float* q_tok, float* q_norm, void* h,
+                               int free_sms, void* ws, size_t ws_bytes,
+                               dspark_stream_t stream);
 
 /*
  * The two halves of one draft position of dspark_draft_sample, for callers

@@ -47,6 +47,8 @@ SIGNATURES = {
                                _sz, _p]),
     "dspark_draft_sample_recurrent": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64,
                                            _u64, _p, _p, _p, _p, _p, _p, _p, _sz, _p]),
+    "dspark_draft_sample_beside": (_i, [_p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64,
+                                        _u64, _p, _p, _p, _p, _p, _p, _i, _p, _sz, _p]),
     "dspark_draft_sample_static": (_i, [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _u64, _u64,
                                         _p, _p, _p, _p, _p, _p]),
     "dspark_sts_fit": (_i, [_p, _p, _i, _i, _p, _p, _p, _p, _p, _sz, _p]),
@@ -193,6 +195,32 @@ def draft_sample_recurrent(base, U, W, R, bias_scale, last_tok, temp, seed: int,
         _ptr(q_norm, "q_norm", f32, (B, K, 2), dev), _ptr(h, "h", base.dtype, (B, K, r), dev),
         _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
     _call("dspark_draft_sample_recurrent", dev, args, stream)
+
+
+def draft_sample_beside(base, U, W, R, bias_scale, last_tok, temp, seed: int, round_id: int,
+                        x, d, q_lse, q_tok, h, free_sms: int, ws, stream=None,
+                        q_norm=None) -> None:
+    """dspark_draft_sample_beside: the draft (Markov head when R is None, else
+    the recurrent head with its states in h) leaving free_sms SMs to kernels of
+    other streams; results identical to draft_sample / draft_sample_recurrent."""
+    B, K, V = base.shape
+    r = U.shape[1]
+    dt = _dtype_code(base)
+    dev, f32, i32 = base.device, torch.float32, torch.int32
+    if R is not None and h is None:
+        raise DSparkError("the recurrent head needs h [B,K,r]")
+    args = (
+        _ptr(base, "base", None, (B, K, V), dev), _ptr(U, "U", base.dtype, (V, r), dev),
+        _ptr(W, "W", base.dtype, (r, V), dev), _ptr(R, "R", base.dtype, (r, r), dev),
+        _ptr(bias_scale, "bias_scale", f32, (B,), dev),
+        _ptr(last_tok, "last_tok", i32, (B,), dev), _ptr(temp, "temp", f32, (B,), dev),
+        B, K, V, r, dt, seed, round_id,
+        _ptr(x, "x", i32, (B, K), dev), _ptr(d, "d", base.dtype, (B, K, V), dev),
+        _ptr(q_lse, "q_lse", f32, (B, K), dev), _ptr(q_tok, "q_tok", f32, (B, K), dev),
+        _ptr(q_norm, "q_norm", f32, (B, K, 2), dev),
+        _ptr(h if R is not None else None, "h", base.dtype, (B, K, r), dev), int(free_sms),
+        _ptr(ws, "ws", None, None, dev), ws.numel() * ws.element_size())
+    _call("dspark_draft_sample_beside", dev, args, stream)
 
 
 def draft_logits(base, U, W, bias_scale, last_tok, x, temp, k: int, d, ws, stream=None) -> None:

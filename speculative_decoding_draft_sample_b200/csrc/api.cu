@@ -19,7 +19,7 @@ using namespace dspark;
 
 namespace {
 
-constexpr int kAbiVersion = (3 << 16) | 0;
+constexpr int kAbiVersion = (3 << 16) | 1;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -176,6 +176,20 @@ cudaError_t launch_logits(const DraftArgs& a, int k, int sms, cudaStream_t s) {
   return draft_tc_supported(a) ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
 }
 
+// All K positions: one cooperative launch for the whole block when the
+// tensor-core path applies and every M-tile gets its own CTAs (free_sms SMs
+// left to other streams); otherwise two launches per position (the same
+// kernels, so the results are identical).
+int draft_run(const DraftArgs& a, int sms, int free_sms, cudaStream_t s) {
+  if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, free_sms, s));
+  for (int k = 1; k <= a.K; ++k) {
+    cudaError_t e = launch_logits(a, k, sms, s);
+    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
+    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  }
+  return DSPARK_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -190,17 +204,7 @@ int dspark_draft_sample(const void* base, const void* U, const void* W, const fl
   if (int e = draft_prepare(a, &sms, true, true, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
                             dtype, seed, round_id, x, d, q_lse, q_tok, q_norm, ws, ws_bytes))
     return e;
-  cudaStream_t s = (cudaStream_t)stream;
-  // one cooperative launch for the whole block when the tensor-core path
-  // applies and every M-tile gets its own CTAs; otherwise two launches per
-  // position (the same kernels, so the results are identical)
-  if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, s));
-  for (int k = 1; k <= K; ++k) {
-    cudaError_t e = launch_logits(a, k, sms, s);
-    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
-    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
-  }
-  return DSPARK_OK;
+  return draft_run(a, sms, kDraftFreeSms, (cudaStream_t)stream);
 }
 
 int dspark_draft_sample_recurrent(const void* base, const void* U, const void* W, const void* R,
@@ -218,16 +222,29 @@ int dspark_draft_sample_recurrent(const void* base, const void* U, const void* W
     return e;
   a.R = R;
   a.H = h;
-  cudaStream_t s = (cudaStream_t)stream;
   // the same launches as dspark_draft_sample; the draw of every position also
   // forms the next position's state, and the bias rows come from the states
-  if (draft_round_tc_supported(a, sms)) return cuda_status(draft_round_tc_launch(a, sms, s));
-  for (int k = 1; k <= K; ++k) {
-    cudaError_t e = launch_logits(a, k, sms, s);
-    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
-    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  return draft_run(a, sms, kDraftFreeSms, (cudaStream_t)stream);
+}
+
+int dspark_draft_sample_beside(const void* base, const void* U, const void* W, const void* R,
+                               const float* bias_scale, const int32_t* last_tok, const float* temp,
+                               int B, int K, int V, int r, int dtype, uint64_t seed,
+                               uint64_t round_id, int32_t* x, void* d, float* q_lse, float* q_tok,
+                               float* q_norm, void* h, int free_sms, void* ws, size_t ws_bytes,
+                               dspark_stream_t stream) {
+  if (free_sms < 0) return DSPARK_ERR_INVALID_ARG;
+  if (R && (!h || !aligned16(R) || !aligned16(h) || r % 8 != 0)) return DSPARK_ERR_INVALID_ARG;
+  DraftArgs a;
+  int sms = 0;
+  if (int e = draft_prepare(a, &sms, true, true, base, U, W, bias_scale, last_tok, temp, B, K, V, r,
+                            dtype, seed, round_id, x, d, q_lse, q_tok, q_norm, ws, ws_bytes))
+    return e;
+  if (R) {
+    a.R = R;
+    a.H = h;
   }
-  return DSPARK_OK;
+  return draft_run(a, sms, free_sms, (cudaStream_t)stream);
 }
 
 int dspark_draft_logits(const void* base, const void* U, const void* W, const float* bias_scale,

@@ -44,7 +44,6 @@ namespace dspark {
 namespace tc {
 
 constexpr int kThreads = 384;      // 4 role warps + 8 epilogue warps
-constexpr int kFreeSms = 2;        // SMs the one-launch round leaves to other streams
 constexpr int kTileM = 128;
 constexpr int kTileN = 256;
 constexpr int kWRows = 64;          // Markov ranks per W stage
@@ -143,11 +142,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
       " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(su32(dst)),
       "l"(map), "r"(su32(bar)), "r"(x), "r"(y), "r"(z), "l"(pol)
       : "memory");
-}
-// Pulls a W box into L2 ahead of its shared-memory load (no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
-               : "memory");
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
                                              int z, uint64_t pol) {
@@ -320,19 +314,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(dst + vb * kWBoxBytes, &map_w, n0 + (kb / kbh) * kWCols + vb * 64,
                       (kb % kbh) * kWRows, &w_full[s], pol_w);
         last[s] = it;
-        // the stage one ring-depth ahead goes to L2 now, so that its load
-        // (issued once a slot frees) is an L2 hit
-        {
-          const int it2 = it + kWStages;
-          const int t2 = it2 / kblocks;
-          if (t2 < n_my * npos) {
-            const int n2 = (nt0 + (t2 % n_my) * nstride) * kTileN;
-            const int kb2 = it2 % kblocks;
-#pragma unroll
-            for (int vb = 0; vb < 2; ++vb)
-              tma_prefetch_2d(&map_w, n2 + (kb2 / kbh) * kWCols + vb * 64, (kb2 % kbh) * kWRows);
-          }
-        }
       }
       if (stop) break;
     }
@@ -528,7 +509,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
     };
     // The recurrent head's next states h_{kq+1} of the rows this CTA drew at
-    // position kq, by its 256 epilogue threads (thread t: output t): R goes
+    // position kq (rows blockIdx.x + j * gridDim.x, j = 0, 1, ..., four at a
+    // time), by its 256 epilogue threads (thread t: output t): R goes
     // through the A buffer, which holds nothing between the position's last
     // MMA and the next gather, in halves of 128 rows; up to four drawn rows'
     // states h_kq at a time sit in the row-statistics buffer. The sums run in
@@ -543,12 +525,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint16_t* Hm = static_cast<uint16_t*>(p.da.H);
       uint16_t* sR = reinterpret_cast<uint16_t*>(sA);      // [128][r]
       uint16_t* sh = reinterpret_cast<uint16_t*>(xstat);   // [4][256]
-      for (int w0 = 0; w0 < 8; w0 += 4) {
+      // the trip count depends only on the grid and B: every epilogue thread
+      // takes the same named barriers
+      for (int w0 = 0; blockIdx.x + (long long)w0 * gridDim.x < p.B; w0 += 4) {
         int rows[4];
         int nr = 0;
         for (int g = 0; g < 4; ++g) {
-          const int rr = blockIdx.x + (w0 + g) * gridDim.x;
-          rows[g] = rr < p.B ? rr : -1;
+          const long long rr = blockIdx.x + (long long)(w0 + g) * gridDim.x;
+          rows[g] = rr < p.B ? (int)rr : -1;
           if (rr < p.B) ++nr;
         }
         if (nr == 0) break;
@@ -897,10 +881,10 @@ cudaError_t draft_logits_tc_launch(const DraftArgs& a, int k, int num_sms, cudaS
 }
 
 bool draft_round_tc_supported(const DraftArgs& a, int num_sms) {
-  return draft_tc_supported(a) && (a.B + tc::kTileM - 1) / tc::kTileM <= num_sms - tc::kFreeSms;
+  return draft_tc_supported(a) && (a.B + tc::kTileM - 1) / tc::kTileM <= num_sms - kDraftFreeSms;
 }
 
-cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t s) {
+cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, int free_sms, cudaStream_t s) {
   using namespace tc;
   CUtensorMap mw, mb, md;
   Params p;
@@ -916,9 +900,11 @@ cudaError_t draft_round_tc_launch(const DraftArgs& a, int num_sms, cudaStream_t 
   p.gbar = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(a.status) + kGridBarrierOffset);
   e = cudaMemsetAsync(p.gbar, 0, sizeof(unsigned int), s);
   if (e != cudaSuccess) return e;
-  // kFreeSms SMs stay free for work on other streams (the prefix schedule,
-  // which needs none of the draft's outputs, runs there at the same time)
-  const int per_m = max(1, (num_sms - kFreeSms) / p.m_tiles);
+  // free_sms SMs stay free for work on other streams (the prefix schedule and
+  // the target rows' statistics need none of the draft's outputs and run there
+  // at the same time); every M-tile keeps at least one CTA
+  const int free_eff = min(max(free_sms, 0), num_sms - p.m_tiles);
+  const int per_m = max(1, (num_sms - free_eff) / p.m_tiles);
   p.m_first = 0;
   p.m_per_launch = p.m_tiles;
   p.ctas_per_m = per_m;

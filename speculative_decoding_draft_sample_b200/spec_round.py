@@ -7,11 +7,45 @@ memory are copied in, the round runs, and the emitted tokens come back.
 """
 from __future__ import annotations
 
+import math
 from typing import Dict, Optional
 
 import torch
 
 from . import binding as bn
+
+# Most SMs a round's draft leaves to the side stream, and how much longer the
+# draft may get for it (the ratio of the most vocabulary tiles per CTA to the
+# most with the library's default of 2 free SMs).
+MAX_FREE_SMS = 20
+FREE_SMS_SLACK = 8.0 / 7.0
+DEFAULT_FREE_SMS = 2
+
+
+def draft_tiles_per_cta(num_sms: int, B: int, V: int, free_sms: int) -> int:
+    """The most 128 x 256 (requests x vocabulary) tiles one CTA of the one-launch
+    draft streams per position when free_sms SMs are left free: each group of
+    128 requests gets (SMs - free) / groups CTAs, which split the vocabulary's
+    256-entry tiles among them."""
+    m = (B + 127) // 128
+    n = (V + 255) // 256
+    free = min(max(free_sms, 0), num_sms - m)
+    per_m = max(1, (num_sms - free) // m)
+    return -(-n // per_m)
+
+
+def beside_free_sms(num_sms: int, B: int, V: int) -> int:
+    """SMs a round's draft leaves to the target rows' statistics on the side
+    stream: the largest count up to MAX_FREE_SMS whose most tiles per CTA stays
+    within FREE_SMS_SLACK of the default's. At B = 256, V = 129280 on 148 SMs
+    that is 20 (eight tiles per CTA instead of seven); where the extra SMs cost
+    no tile (one group of requests over a larger vocabulary) it is the cap."""
+    limit = math.floor(draft_tiles_per_cta(num_sms, B, V, DEFAULT_FREE_SMS) * FREE_SMS_SLACK + 1e-9)
+    best = DEFAULT_FREE_SMS
+    for f in range(DEFAULT_FREE_SMS, MAX_FREE_SMS + 1):
+        if draft_tiles_per_cta(num_sms, B, V, f) <= limit:
+            best = f
+    return best
 
 
 class SpecRound:
@@ -39,6 +73,9 @@ class SpecRound:
         if nbytes == 0:
             raise bn.DSparkError(f"unsupported round shape B={B} K={K} V={V} r={r}")
         self.ws = torch.zeros((nbytes,), dtype=torch.uint8, device=dev)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count if dev.type == "cuda" else 148
+        # SMs the draft leaves to the side stream's statistics when a round has one
+        self.free_sms = beside_free_sms(sms, B, V)
 
     def run(self, inp: Dict[str, torch.Tensor], seed: int, round_id: int,
             mode: int = bn.CUT_COST, threshold: float = 0.0, stream=None,
@@ -47,9 +84,10 @@ class SpecRound:
 
         The prefix schedule needs only the confidence logits, and the target
         rows' statistics only the target logits and the cut, so with a
-        ``side_stream`` both run there, concurrently with the draft (the
-        one-launch draft kernel leaves SMs free for them); the rest of
-        verification waits for both. The calls share the workspace: the draft's
+        ``side_stream`` both run there, concurrently with the draft, which then
+        leaves ``self.free_sms`` SMs free for them (dspark_draft_sample_beside;
+        the same results as dspark_draft_sample); the rest of verification
+        waits for both. The calls share the workspace: the draft's
         partials and the statistics occupy different regions of it, and they
         meet only in its status block, which every call updates atomically.
         """
@@ -69,10 +107,16 @@ class SpecRound:
             side_stream.wait_event(fork)
             schedule_and_stats(side_stream)
             join.record(side_stream)
-        if inp.get("R") is not None:  # the recurrent head; its states land in self.h
-            if self.h is None:
-                self.h = torch.empty((self.B, self.K, self.r), dtype=self.dtype, device=self.x.device)
-            bn.draft_sample_recurrent(inp["base"], inp["U"], inp["W"], inp["R"],
+        R = inp.get("R")
+        if R is not None and self.h is None:  # the recurrent head; its states land in self.h
+            self.h = torch.empty((self.B, self.K, self.r), dtype=self.dtype, device=self.x.device)
+        if side_stream is not None:
+            bn.draft_sample_beside(inp["base"], inp["U"], inp["W"], R, inp.get("bias_scale"),
+                                   inp["last_tok"], inp["temp"], seed, round_id, self.x, self.d,
+                                   self.q_lse, self.q_tok, self.h, self.free_sms, self.ws, main,
+                                   q_norm=self.q_norm)
+        elif R is not None:
+            bn.draft_sample_recurrent(inp["base"], inp["U"], inp["W"], R,
                                       inp.get("bias_scale"), inp["last_tok"], inp["temp"], seed,
                                       round_id, self.x, self.d, self.q_lse, self.q_tok, self.h,
                                       self.ws, main, q_norm=self.q_norm)

@@ -41,6 +41,15 @@ int main(void) {
   CHECK(dspark_draft_sample(NULL, NULL, NULL, NULL, i32, f32, 4, 4, 1024, 16, DSPARK_F32, 1, 0,
                             i32, NULL, f32, f32, NULL, ws, sizeof ws, NULL) ==
         DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_draft_sample_beside(NULL, NULL, NULL, NULL, NULL, i32, f32, 4, 4, 1024, 16,
+                                   DSPARK_F32, 1, 0, i32, NULL, f32, f32, NULL, NULL, 20, ws,
+                                   sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
+  CHECK(dspark_draft_sample_beside(f32, f32, f32, NULL, NULL, i32, f32, 4, 4, 1024, 16,
+                                   DSPARK_F32, 1, 0, i32, f32, f32, f32, NULL, NULL, -1, ws,
+                                   sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG); /* free_sms < 0 */
+  CHECK(dspark_draft_sample_beside(f32, f32, f32, f32, NULL, i32, f32, 4, 4, 1024, 16,
+                                   DSPARK_F32, 1, 0, i32, f32, f32, f32, NULL, NULL, 2, ws,
+                                   sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG); /* R without h */
   CHECK(dspark_prefix_schedule(NULL, f32, f32, 0.f, 4, 1, DSPARK_CUT_COST, 0.f, i32, f32, ws,
                                sizeof ws, NULL) == DSPARK_ERR_INVALID_ARG);
   CHECK(dspark_prefix_schedule(f32, f32, f32, 0.f, 4, 65, DSPARK_CUT_COST, 0.f, i32, f32, ws,

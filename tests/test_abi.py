@@ -58,6 +58,8 @@ def test_workspace_sizes(lib):
 def test_null_pointers_rejected_before_any_device_call(lib):
     p = ctypes.c_void_p(0)
     assert lib.dspark_draft_sample(p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p, p, p, 0, p) == -1
+    assert lib.dspark_draft_sample_beside(p, p, p, p, p, p, p, 4, 4, 1024, 16, 0, 1, 0, p, p, p, p,
+                                          p, p, 20, p, 0, p) == -1
     assert lib.dspark_verify(p, p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0, p) == -1
     assert lib.dspark_verify_from_stats(p, p, p, p, p, p, p, 4, 4, 1024, 0, 1, 0, p, p, p, p, 0,
                                         p) == -1

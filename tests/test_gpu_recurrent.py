@@ -25,6 +25,9 @@ CASES = [
     wl.scaled(wl.STRESS, name="rnn_stress_small", B=200, K=8, V=2056),              # two M-tiles, greedy mix
     wl.scaled(wl.DSPARK5, name="rnn_f32_small", B=12, V=3000 // 8 * 8, dtype=wl.F32, r=32),  # CUDA-core path
     wl.scaled(wl.DSPARK5, name="rnn_bf16_r512", B=10, K=3, V=2048, r=512),          # CUDA-core path, bf16
+    # one-launch path with more drawn rows per CTA than its eight drawing warps
+    # (10 groups of 128 requests on 140 CTAs: rows past 8 x 140 = 1120)
+    wl.scaled(wl.DSPARK5, name="rnn_many_rows", B=1200, K=3, V=2048),
 ]
 
 
