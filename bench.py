@@ -388,8 +388,11 @@ def main():
     emit_all = replicas.sum_over_ranks(float(emitted), "cuda")
     rounds_per_s = world * 1000.0 / ms
 
-    # per-stage times (same stream, CUDA events), each stage alone
+    # per-stage times (same stream, CUDA events), each stage alone; the NVTX
+    # range lets a profiler select these launches (ncu --nvtx --nvtx-include
+    # stage_timing/), e.g. the full-width draft kernel the roofline times
     s_bytes = w.nbytes_per_logit
+    torch.cuda.nvtx.range_push("stage_timing")
     with torch.cuda.stream(stream):
         if args.head == "recurrent":
             ms_draft = time_region(lambda: bn.draft_sample_recurrent(
@@ -414,6 +417,8 @@ def main():
             dev["target"], rnd.d, rnd.x, rnd.q_tok, rnd.cut, dev["temp"], wl.PHILOX_SEED,
             round_id, rnd.accepted, rnd.out, rnd.n_emit, rnd.ws, stream, q_norm=rnd.q_norm),
             stream, 20)
+
+    torch.cuda.nvtx.range_pop()
 
     # verification's algorithmic bytes (the survey's count): target rows 0..cut[b]
     # of every request, plus draft row a_b of every request rejected before its
