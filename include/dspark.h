@@ -375,7 +375,7 @@ int dspark_sts_fit(const float* conf_logit, const uint8_t* survived, int N, int 
  * only input and output buffers, and latency-critical paths that cannot accept
  * cudaMalloc's implicit synchronisation have no way to provide one.
  *
- * Same arguments, computation and results as dspark_draft_sample, without
+ * Same arguments, computation, launches and results as dspark_draft_sample, without
  * ws/ws_bytes and without the optional q_norm output (dspark_verify then
  * recomputes the draft rows' normalisers). The scratch is a fixed 8 MiB array inside the library's device
  * image, held on every GPU that loads the library until the process exits; the

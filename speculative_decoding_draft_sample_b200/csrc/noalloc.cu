@@ -121,11 +121,18 @@ extern "C" int dspark_draft_sample_static(const void* base, const void* U, const
   a.H = nullptr;
   a.partials = reinterpret_cast<float2*>(static_cast<char*>(scratch) + kStatusBytes);
   a.nchunk = nchunk;
-  const bool tc = draft_tc_supported(a);
-  for (int k = 1; k <= K; ++k) {
-    cudaError_t e = tc ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
-    if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
-    if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+  // the launches of dspark_draft_sample: one cooperative launch for the whole
+  // block where the tensor-core path applies (its grid-barrier counter lives
+  // in the status block, which the scratch holds too), else two per position
+  if (draft_round_tc_supported(a, sms)) {
+    if (draft_round_tc_launch(a, sms, kDraftFreeSms, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  } else {
+    const bool tc = draft_tc_supported(a);
+    for (int k = 1; k <= K; ++k) {
+      cudaError_t e = tc ? draft_logits_tc_launch(a, k, sms, s) : draft_logits_simt_launch(a, k, s);
+      if (e == cudaSuccess) e = draft_sample_launch(a, k, s);
+      if (e != cudaSuccess) return DSPARK_ERR_CUDA;
+    }
   }
   if (status_out) {
     copy_status<<<1, 1, 0, s>>>(a.status, status_out);
