@@ -315,7 +315,9 @@ int dspark_verify(const void* target, const void* d, const int32_t* x,
  *   (all K + 1 rows when cut is NULL), the softmax partials of every 2 KB
  *   chunk of the row, (max z, sum 2^(z - max z)) of z = target * log2(e) /
  *   temp[b], or (max, lowest argmax) for temp[b] == 0, written to the
- *   workspace's statistics region. The region lies past the draft's partials
+ *   workspace's statistics region, and (with a cut) the order in which the
+ *   final kernel takes the requests (cut descending, index ascending) after
+ *   it. The statistics region lies past the draft's partials
  *   of a workspace of the same size, so this call may run on another stream
  *   concurrently with dspark_draft_sample on that workspace; it must complete
  *   before dspark_verify_from_stats starts (an event or the same stream).

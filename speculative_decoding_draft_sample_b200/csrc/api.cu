@@ -19,7 +19,7 @@ using namespace dspark;
 
 namespace {
 
-constexpr int kAbiVersion = (3 << 16) | 1;
+constexpr int kAbiVersion = (3 << 16) | 2;
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -29,6 +29,7 @@ inline int nchunks(int V) { return (V + kChunk - 1) / kChunk; }
 
 // Workspace layout shared by the calls of one round:
 //   [status block 256][draft chunk partials][target-row statistics][work counter 256]
+//   [verification order: B request indices]
 // The statistics sit past the draft's partials, so that dspark_verify_target_stats
 // may run on another stream while dspark_draft_sample runs (they share only the
 // status block, which both update atomically).
@@ -40,6 +41,7 @@ inline size_t stats_offset(int B, int V) { return kStatusBytes + draft_region(B,
 inline size_t counter_offset(int B, int K, int V, int dtype) {
   return stats_offset(B, V) + stats_region(B, K, V, dtype);
 }
+inline size_t order_offset(int B, int K, int V, int dtype) { return counter_offset(B, K, V, dtype) + 256; }
 
 bool shape_ok(int B, int K, int V, int dtype) {
   if (dtype != DSPARK_F32 && dtype != DSPARK_BF16) return false;
@@ -103,7 +105,7 @@ size_t dspark_workspace_bytes(int op, int B, int K, int V, int r, int dtype) {
       return calib_workspace_bytes(B, K);
     case DSPARK_OP_VERIFY:
       if (!shape_ok(B, K, V, dtype)) return 0;
-      return counter_offset(B, K, V, dtype) + 256;
+      return order_offset(B, K, V, dtype) + round_up((size_t)B * sizeof(int32_t), 256);
     default:
       return 0;
   }
@@ -324,6 +326,7 @@ int stats_prepare(StatsArgs& sa, int* sms, const void* target, const int32_t* cu
   sa.partials = reinterpret_cast<float2*>(w + stats_offset(B, V));
   sa.nchunk = stats_chunks(V, dtype);
   sa.next = reinterpret_cast<unsigned long long*>(w + counter_offset(B, K, V, dtype));
+  sa.order = reinterpret_cast<int32_t*>(w + order_offset(B, K, V, dtype));
   sa.status = static_cast<Status*>(ws);
   return DSPARK_OK;
 }
@@ -362,6 +365,7 @@ int verify_decide(const void* target, const void* d, const int32_t* x, const flo
   a.status = static_cast<Status*>(ws);
   a.stats = sa.partials;
   a.nstat = sa.nchunk;
+  a.order = cut ? sa.order : nullptr;  // written by the statistics pass
   const int C = verify_cluster_size(B, V, dtype, sms);
   return cuda_status(verify_launch(a, C, s));
 }

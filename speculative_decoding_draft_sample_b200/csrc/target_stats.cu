@@ -81,6 +81,38 @@ __device__ __forceinline__ float warp_max_nan_all(float v) {
 
 }  // namespace
 
+// The order in which verification takes the requests: cut descending, index
+// ascending (the longest chains of rows first), by one warp: a histogram of
+// the clamped cuts, the start of every cut value's range, then every request's
+// place, 32 requests at a time (peers with the same cut keep index order).
+__device__ void write_order(const StatsArgs& a, int lane, int* cnt) {
+  const int K = a.K;
+  for (int v = lane; v <= K; v += 32) cnt[v] = 0;
+  __syncwarp();
+  for (int i = lane; i < a.B; i += 32) atomicAdd(&cnt[min(max(a.cut[i], 0), K)], 1);
+  __syncwarp();
+  if (lane == 0) {  // cnt[v] becomes the first place of cut value v
+    int base = 0;
+    for (int v = K; v >= 0; --v) {
+      const int c = cnt[v];
+      cnt[v] = base;
+      base += c;
+    }
+  }
+  __syncwarp();
+  const unsigned below = (1u << lane) - 1u;
+  for (int i0 = 0; i0 < a.B; i0 += 32) {
+    const int i = i0 + lane;
+    const int L = (i < a.B) ? min(max(a.cut[i], 0), K) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, L);
+    const int rank = __popc(peers & below);
+    if (L >= 0) a.order[cnt[L] + rank] = i;
+    __syncwarp();
+    if (L >= 0 && rank == 0) cnt[L] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 template <int DT>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm) target_stats_kernel(StatsArgs a) {
   extern __shared__ __align__(128) unsigned char ring_raw[];
@@ -89,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) target_stats_kernel(Stat
   __shared__ __align__(8) uint64_t empty[kSlots];
   __shared__ int4 meta[kSlots];  // (request, row, segment, bytes); request < 0 ends the stream
   __shared__ int dead;
+  __shared__ int ord_cnt[65];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int es = Elem<DT>::kBytes;
@@ -109,6 +142,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) target_stats_kernel(Stat
 
   if (warp == kConsumers) {
     // ---------------- producer ----------------
+    if (blockIdx.x == 0 && a.cut && a.order) write_order(a, lane, ord_cnt);
+    __syncwarp();
     if (lane == 0) {
       const char* target = static_cast<const char*>(a.target);
       uint32_t u = 0;             // units (row segments) issued

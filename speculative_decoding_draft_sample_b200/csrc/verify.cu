@@ -570,11 +570,13 @@ __device__ __forceinline__ float2 combine_ranks(const Exch* got, int C) {
 // Cluster q verifies the request of rank q in the order (cut descending,
 // index ascending): the longest chains of rows start in the first wave of
 // clusters and the requests that verify a single row take the slots that free
-// up last. Every CTA of the cluster computes the same answer: a histogram of
-// the (clamped) cuts, the cut value whose range holds q, then the position of
-// the request among those with that cut, in index order.
+// up last. The statistics pass writes this order once (a.order); without it
+// every CTA of the cluster computes the same answer: a histogram of the
+// (clamped) cuts, the cut value whose range holds q, then the position of the
+// request among those with that cut, in index order.
 __device__ int request_of(const VerifyArgs& a, int q, int* cnt, int* s_req) {
   if (!a.cut) return q;
+  if (a.order) return a.order[q];  // the same order, made once by the statistics pass
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int K = a.K;
   for (int v = tid; v <= K; v += kVThreads) cnt[v] = 0;

@@ -18,6 +18,7 @@ struct StatsArgs {
   float2* partials;          // [B, K+1, nchunk] chunk partials (rows past the cut untouched)
   int nchunk;                // stats_chunks(V, dtype)
   unsigned long long* next;  // work counter, zeroed by the launcher
+  int32_t* order;            // [B] out: the verification order (cut descending, index ascending)
   Status* status;
 };
 
@@ -42,6 +43,7 @@ struct VerifyArgs {
   int slice;              // vocabulary entries per CTA (multiple of 8)
   const float2* stats;    // [B, K+1, nstat] target-row partials from target_stats
   int nstat;              // stats_chunks(V, dtype)
+  const int32_t* order;   // [B] from target_stats, or null (index order)
 };
 
 // CTAs per request (the cluster size) for this batch shape.

@@ -26,9 +26,10 @@ int main(void) {
   /* draft: status block + one (max, sum) pair per request and 256-entry chunk */
   CHECK(dspark_workspace_bytes(DSPARK_OP_DRAFT, 256, 5, 129280, 256, DSPARK_BF16) ==
         256 + (size_t)256 * 505 * 8);
-  /* verify: status block, the draft's partials, per-chunk target-row statistics, a counter */
+  /* verify: status block, the draft's partials, per-chunk target-row statistics, a counter,
+     the verification order */
   CHECK(dspark_workspace_bytes(DSPARK_OP_VERIFY, 256, 5, 129280, 256, DSPARK_BF16) ==
-        256 + (size_t)256 * 505 * 8 + (size_t)256 * 6 * 127 * 8 + 256);
+        256 + (size_t)256 * 505 * 8 + (size_t)256 * 6 * 127 * 8 + 256 + 1024);
   CHECK(dspark_workspace_bytes(DSPARK_OP_SCHEDULE, 1024, 8, 0, 0, 0) == 256);
   CHECK(dspark_workspace_bytes(DSPARK_OP_DRAFT, 4, 4, 1001, 16, DSPARK_F32) == 0); /* V % 8 */
   CHECK(dspark_workspace_bytes(DSPARK_OP_VERIFY, 4, 65, 1024, 16, DSPARK_F32) == 0); /* K > 64 */

@@ -42,9 +42,9 @@ def test_workspace_sizes(lib):
     assert bn.workspace_bytes(bn.OP_DRAFT, 256, 5, 129280, 256, bn.BF16) == 256 + 256 * 505 * 8
     # verify: status block, the draft's partials (disjoint, so the target statistics
     # can be made beside the draft), (max, sum) per request, target row and 2 KB
-    # chunk of rows 0..K, the work counter
+    # chunk of rows 0..K, the work counter, the verification order (4 bytes per request)
     assert bn.workspace_bytes(bn.OP_VERIFY, 256, 5, 129280, 256, bn.BF16) == \
-        256 + 256 * 505 * 8 + 256 * 6 * 127 * 8 + 256
+        256 + 256 * 505 * 8 + 256 * 6 * 127 * 8 + 256 + 1024
     assert bn.workspace_bytes(bn.OP_SCHEDULE, 1024, 8, 0, 0, 0) == 256
     assert bn.workspace_bytes(bn.OP_SCHEDULE, 1024, 65, 0, 0, 0) == 0  # K > 64
     assert bn.workspace_bytes(bn.OP_DRAFT, 4, 4, 1001, 16, bn.F32) == 0  # V % 8
