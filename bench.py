@@ -8,7 +8,9 @@ temperatures {0.6, 0.8, 1.0}, a cost table with a step at 512 verified tokens.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
 Under torchrun every rank runs its own batch (different seed) with no
-collective on the data path (weak scaling); timing is bracketed by a barrier
+collective on the data path (weak scaling; with --global-schedule one prefix
+cut spans every rank's requests, after an all-gather of their confidence
+logits); timing is bracketed by a barrier
 and synchronisation, taken with CUDA events, and reduced with MAX over ranks.
 Prints one JSON line on rank 0.
 """
@@ -30,8 +32,8 @@ sys.path.insert(0, ROOT)
 from speculative_decoding_draft_sample_b200 import binding as bn  # noqa: E402
 from speculative_decoding_draft_sample_b200 import replicas  # noqa: E402
 from speculative_decoding_draft_sample_b200 import workloads as wl  # noqa: E402
-from speculative_decoding_draft_sample_b200.spec_round import (DEVICE_KEYS, SpecRound,  # noqa: E402
-                                                                run_host, to_device)
+from speculative_decoding_draft_sample_b200.spec_round import (DEVICE_KEYS, GlobalSchedule,  # noqa: E402
+                                                                SpecRound, run_host, to_device)
 
 METRIC = "spec rounds/s & accepted tok/s at B=256,K=5,V=129280; verify HBM GB/s vs peak"
 UNIT = "rounds/s"
@@ -309,6 +311,9 @@ def main():
                     help="survival threshold of --cut threshold")
     ap.add_argument("--head", default="markov", choices=["markov", "recurrent"],
                     help="sequential draft head: the Markov head (default) or the recurrent one")
+    ap.add_argument("--global-schedule", action="store_true",
+                    help="one prefix schedule over every rank's requests (an all-gather of the "
+                         "confidence logits) instead of one per engine")
     args = ap.parse_args()
     if args.load_sweep:
         load_sweep()
@@ -338,8 +343,15 @@ def main():
     mode = CUT_MODES[args.cut]
     threshold = args.threshold if mode == bn.CUT_THRESHOLD else 0.0
 
+    # optionally one cut over every rank's requests, against the combined batch's cost table
+    gsched = None
+    if args.global_schedule:
+        step_cost_g, fixed_g = wl.cost_table(w, w.B * world)
+        gsched = GlobalSchedule(w.B, w.K, step_cost_g, fixed_g, rank, world)
+
     def step():
-        rnd.run(dev, wl.PHILOX_SEED, round_id, mode, threshold, stream=stream, side_stream=side)
+        rnd.run(dev, wl.PHILOX_SEED, round_id, mode, threshold, stream=stream, side_stream=side,
+                global_schedule=gsched)
 
     with torch.cuda.stream(stream):
         step()
@@ -447,12 +459,13 @@ def main():
     with torch.cuda.stream(stream):
         for _ in range(2):
             run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h, mode, stream=stream,
-                     side_stream=side, threshold=threshold)
+                     side_stream=side, threshold=threshold, global_schedule=gsched)
         replicas.barrier()
         e2e_steps = max(3, args.steps // 5)
         ms_e2e = time_region(lambda: run_host(rnd, host, dev, wl.PHILOX_SEED, round_id, out_h, n_h,
                                               mode, stream=stream, side_stream=side,
-                                              threshold=threshold), stream, e2e_steps)
+                                              threshold=threshold, global_schedule=gsched),
+                                     stream, e2e_steps)
     ms_e2e = replicas.max_over_ranks(ms_e2e, "cuda")
 
     in_bytes = (w.B * (w.K + 1) * w.V + w.B * w.K * w.V + 2 * w.V * w.r) * s_bytes
@@ -473,6 +486,7 @@ def main():
         "data": "synthetic (seeded Zipf+noise logits, random Markov factors)",
         "config": {"workload": w.name, "B": w.B, "K": w.K, "V": w.V, "r": w.r,
                    "global_batch": w.B * world, "parallelism": f"replicas{world}",
+                   "schedule": "global" if gsched is not None else "per-engine",
                    "cut": args.cut + (f" {threshold}" if mode == bn.CUT_THRESHOLD else ""),
                    "head": args.head,
                    "l2": (f"inputs ({in_bytes / 1e6:.0f} MB) larger than L2 (126 MB); not flushed"

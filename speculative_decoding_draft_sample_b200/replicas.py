@@ -1,10 +1,13 @@
-"""Host-side logic of running the round on several GPUs as independent replicas.
+"""Host-side logic of running the round on several GPUs.
 
-Requests are independent through drafting and verification and the prefix cut
-is per engine (every GPU schedules its own batch against its own cost table),
-so N GPUs run N independent batches with no collective on the data path
-(weak scaling). The only collectives are the timing bookkeeping: a barrier
-around the timed region and MAX / SUM reductions of per-rank numbers.
+Requests are independent through drafting and verification, and by default
+the prefix cut is per engine (every GPU schedules its own batch against its
+own cost table), so N GPUs run N independent batches with no collective on the
+data path (weak scaling); the only collectives are then the timing
+bookkeeping: a barrier around the timed region and MAX / SUM reductions of
+per-rank numbers. Optionally one schedule spans every GPU's requests
+(spec_round.GlobalSchedule): its single data-path collective is the
+all-gather of the confidence logits, all_gather_rows below.
 """
 from __future__ import annotations
 
@@ -57,6 +60,16 @@ def max_over_ranks(v: float, device="cpu") -> float:
 
 def sum_over_ranks(v: float, device="cpu") -> float:
     return _reduce(v, dist.ReduceOp.SUM, device)
+
+
+def all_gather_rows(t: torch.Tensor) -> torch.Tensor:
+    """Every rank's t (same shape on every rank) stacked along dim 0 in rank
+    order; t itself when there is one rank. Runs on the current stream."""
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return t
+    parts = [torch.empty_like(t) for _ in range(dist.get_world_size())]
+    dist.all_gather(parts, t.contiguous())
+    return torch.cat(parts, 0)
 
 
 def barrier() -> None:

@@ -8,11 +8,12 @@ memory are copied in, the round runs, and the emitted tokens come back.
 from __future__ import annotations
 
 import math
-from typing import Dict, Optional
+from typing import Callable, Dict, Optional
 
 import torch
 
 from . import binding as bn
+from . import replicas
 
 # Most SMs a round's draft leaves to the side stream, and how much longer the
 # draft may get for it (the ratio of the most vocabulary tiles per CTA to the
@@ -48,6 +49,48 @@ def beside_free_sms(num_sms: int, B: int, V: int) -> int:
     return best
 
 
+class GlobalSchedule:
+    """One prefix schedule over the requests of every rank, in place of one
+    per engine: the confidence logits of all ranks are gathered (the only
+    data-path collective), every rank runs the same schedule on the combined
+    batch against the combined batch's cost table, so all ranks compute the
+    same cut, and each keeps the slice of its own requests (rank r holds
+    requests r * B .. r * B + B - 1 of the combined batch).
+
+    step_cost has (B * world) * (K + 1) entries (workloads.cost_table of the
+    combined batch); gather (default replicas.all_gather_rows) stacks every
+    rank's [B, K] confidence logits in rank order.
+    """
+
+    def __init__(self, B: int, K: int, step_cost, fixed_cost: float, rank: int, world: int,
+                 device: str = "cuda", gather: Optional[Callable] = None):
+        if not 0 <= rank < world:
+            raise bn.DSparkError(f"rank {rank} outside a world of {world}")
+        self.B, self.K, self.rank, self.world = B, K, rank, world
+        bg = B * world
+        dev = torch.device(device)
+        self.step_cost = torch.as_tensor(step_cost, dtype=torch.float32).to(dev).contiguous()
+        if self.step_cost.numel() != bg * (K + 1):
+            raise bn.DSparkError(f"step_cost needs {bg * (K + 1)} entries for {world} ranks of "
+                                 f"{B} requests, got {self.step_cost.numel()}")
+        self.fixed_cost = float(fixed_cost)
+        self.cut = torch.empty((bg,), dtype=torch.int32, device=dev)
+        self.survival = torch.empty((bg, K), dtype=torch.float32, device=dev)
+        self.gather = gather if gather is not None else replicas.all_gather_rows
+
+    def run(self, conf_logit, pos_temp, mode: int, threshold: float, cut, survival, ws,
+            stream) -> None:
+        """This rank's cut [B] and survival [B, K] from the combined batch's
+        schedule, on `stream` (the schedule kernel's status lands in ws)."""
+        with torch.cuda.stream(stream):
+            conf_all = self.gather(conf_logit)
+            bn.prefix_schedule(conf_all, pos_temp, self.step_cost, self.fixed_cost, mode,
+                               threshold, self.cut, self.survival, ws, stream)
+            lo = self.rank * self.B
+            cut.copy_(self.cut[lo:lo + self.B])
+            survival.copy_(self.survival[lo:lo + self.B])
+
+
 class SpecRound:
     def __init__(self, B: int, K: int, V: int, r: int, dtype: torch.dtype = torch.bfloat16,
                  device: str = "cuda"):
@@ -79,7 +122,7 @@ class SpecRound:
 
     def run(self, inp: Dict[str, torch.Tensor], seed: int, round_id: int,
             mode: int = bn.CUT_COST, threshold: float = 0.0, stream=None,
-            side_stream=None) -> None:
+            side_stream=None, global_schedule: Optional[GlobalSchedule] = None) -> None:
         """Issues the round on ``stream`` (no host synchronisation).
 
         The prefix schedule needs only the confidence logits, and the target
@@ -94,9 +137,13 @@ class SpecRound:
         main = stream if stream is not None else torch.cuda.current_stream(self.x.device)
 
         def schedule_and_stats(s):
-            bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
-                               float(inp["fixed_cost"]), mode, threshold, self.cut, self.survival,
-                               self.ws, s)
+            if global_schedule is not None:  # one cut over every rank's requests
+                global_schedule.run(inp["conf_logit"], inp["pos_temp"], mode, threshold, self.cut,
+                                    self.survival, self.ws, s)
+            else:
+                bn.prefix_schedule(inp["conf_logit"], inp["pos_temp"], inp["step_cost"],
+                                   float(inp["fixed_cost"]), mode, threshold, self.cut,
+                                   self.survival, self.ws, s)
             bn.verify_target_stats(inp["target"], self.cut, inp["temp"], self.ws, s)
 
         if side_stream is not None:
@@ -165,10 +212,11 @@ def to_device(inp: Dict[str, object], device: str = "cuda", pin: bool = False) -
 def run_host(rnd: SpecRound, host: Dict[str, object], dev: Dict[str, object], seed: int,
              round_id: int, out_host: torch.Tensor, n_emit_host: torch.Tensor,
              mode: int = bn.CUT_COST, stream=None, side_stream=None,
-             threshold: float = 0.0) -> None:
+             threshold: float = 0.0, global_schedule: Optional[GlobalSchedule] = None) -> None:
     """End to end from pinned host buffers: H2D copies, the round, D2H of the tokens."""
     for k in DEVICE_KEYS:
         dev[k].copy_(host[k], non_blocking=True)
-    rnd.run(dev, seed, round_id, mode, threshold, stream=stream, side_stream=side_stream)
+    rnd.run(dev, seed, round_id, mode, threshold, stream=stream, side_stream=side_stream,
+            global_schedule=global_schedule)
     out_host.copy_(rnd.out, non_blocking=True)
     n_emit_host.copy_(rnd.n_emit, non_blocking=True)

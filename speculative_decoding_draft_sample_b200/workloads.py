@@ -19,7 +19,7 @@ from __future__ import annotations
 
 import dataclasses
 import os
-from typing import Dict, List, Optional, Sequence
+from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 import torch
@@ -185,7 +185,20 @@ def small_inputs(w: Workload) -> Dict[str, object]:
     bias_scale[kinds["identical"]] = 0.0
     conf_logit = (w.conf_mean + w.conf_std * rng.standard_normal((B, K))).astype(np.float32)
     pos_temp = np.linspace(w.pos_temp_lo, w.pos_temp_hi, K).astype(np.float32)
-    n_slots = B * (K + 1)
+    step_cost, fixed_cost = cost_table(w, B)
+    return dict(U=U, W=W, last_tok=last_tok, temp=temp, bias_scale=bias_scale,
+                conf_logit=conf_logit, pos_temp=pos_temp, step_cost=step_cost,
+                fixed_cost=fixed_cost, identical=kinds["identical"],
+                independent=kinds["independent"])
+
+
+def cost_table(w: Workload, B: int) -> Tuple[np.ndarray, float]:
+    """The workload's cost per verified token, step_cost[n - 1] for the n-th
+    verified token of a batch of B requests (B(K+1) entries), and its fixed
+    cost (B unless the workload sets one: one slot per request is always
+    verified). A schedule over several engines' requests takes the table of
+    their combined batch."""
+    n_slots = B * (w.K + 1)
     n = np.arange(1, n_slots + 1, dtype=np.float64)  # 1-based verified-token count
     if w.cost_kind == "flat":
         step_cost = np.ones(n_slots, np.float32)
@@ -195,11 +208,7 @@ def small_inputs(w: Workload) -> Dict[str, object]:
         step_cost = np.where(n <= w.cost_step_at, 1.0, w.cost_step_hi).astype(np.float32)
     else:
         raise ValueError(w.cost_kind)
-    fixed_cost = float(B if w.fixed_cost is None else w.fixed_cost)
-    return dict(U=U, W=W, last_tok=last_tok, temp=temp, bias_scale=bias_scale,
-                conf_logit=conf_logit, pos_temp=pos_temp, step_cost=step_cost,
-                fixed_cost=fixed_cost, identical=kinds["identical"],
-                independent=kinds["independent"])
+    return step_cost, float(B if w.fixed_cost is None else w.fixed_cost)
 
 
 def recurrent_factor(w: Workload, std: float = 1.0) -> torch.Tensor:
