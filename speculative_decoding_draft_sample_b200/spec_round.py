@@ -18,7 +18,7 @@ from . import replicas
 # Most SMs a round's draft leaves to the side stream, and how much longer the
 # draft may get for it (the ratio of the most vocabulary tiles per CTA to the
 # most with the library's default of 2 free SMs).
-MAX_FREE_SMS = 20
+MAX_FREE_SMS = 32
 FREE_SMS_SLACK = 8.0 / 7.0
 DEFAULT_FREE_SMS = 2
 
@@ -39,8 +39,8 @@ def beside_free_sms(num_sms: int, B: int, V: int) -> int:
     """SMs a round's draft leaves to the target rows' statistics on the side
     stream: the largest count up to MAX_FREE_SMS whose most tiles per CTA stays
     within FREE_SMS_SLACK of the default's. At B = 256, V = 129280 on 148 SMs
-    that is 20 (eight tiles per CTA instead of seven); where the extra SMs cost
-    no tile (one group of requests over a larger vocabulary) it is the cap."""
+    that is 20 (eight tiles per CTA instead of seven); for one group of requests
+    over V = 151936 it is 29 (five tiles per CTA either way)."""
     limit = math.floor(draft_tiles_per_cta(num_sms, B, V, DEFAULT_FREE_SMS) * FREE_SMS_SLACK + 1e-9)
     best = DEFAULT_FREE_SMS
     for f in range(DEFAULT_FREE_SMS, MAX_FREE_SMS + 1):

@@ -33,10 +33,12 @@ def test_choices_at_the_benchmark_shapes():
     assert sr.draft_tiles_per_cta(148, 256, 129280, 2) == 7
     assert sr.beside_free_sms(148, 256, 129280) == 20
     assert sr.draft_tiles_per_cta(148, 256, 129280, 20) == 8
-    # one group over V = 151936 (594 tiles): 5 tiles per CTA with 2 or with 20 free
+    # one group over V = 151936 (594 tiles): 5 tiles per CTA with 2 or with 29 free
+    # (119 CTAs), 6 with 30 free (118 CTAs)
     for B in (64, 128):
-        assert sr.beside_free_sms(148, B, 151936) == 20
-        assert sr.draft_tiles_per_cta(148, B, 151936, 20) == 5
+        assert sr.beside_free_sms(148, B, 151936) == 29
+        assert sr.draft_tiles_per_cta(148, B, 151936, 29) == 5
+        assert sr.draft_tiles_per_cta(148, B, 151936, 30) == 6
     # Stress: 8 groups, 18 CTAs each -> 33 tiles; 12 free -> 17 CTAs -> 35 <= 37;
     # 13 free -> 16 CTAs -> 38 > 37
     assert sr.beside_free_sms(148, 1024, 151936) == 12
